@@ -1,0 +1,365 @@
+#!/usr/bin/env python
+"""Benchmark of the Local-Hessian NVFP4 calibration hot path on B200.
+
+One step = the whole hot path for one layer, every kernel from liblh.so:
+    lh_absmax -> lh_accumulate_hessian -> lh_sweep_scales (126 candidates) -> lh_fake_quant
+over the seeded synthetic layer (default: the attention projection,
+W [4096,4096] bf16, X [2048,4096] bf16; --config picks another).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference] [--config 0..4]
+
+Prints one JSON line (rank 0). `value` is NVFP4 blocks calibrated per second
+of the whole step, summed over ranks (each rank calibrates its own layer: the
+path shards by layer/expert with no collective, weak scaling). Timing: CUDA
+events on the launching stream, L2 flushed before every timed step, max over
+ranks. `--impl reference` times the FP64 CPU oracle on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 blocks swept/sec (126 cands) + Hessian tokens/sec; % of roofline, 1 B200"
+UNIT = "blocks/s"
+SWEEP_FLOP_PER_BLOCK = 126 * 152 * 2   # 16 dw FMA + 136 symmetric-form FMA per candidate
+FP32_LANES_PER_SM = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), sm_max_mhz=float(d.get("sm_max_mhz", 1965.0)), source="measured")
+    return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["unsampled"], samples=0)
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(mx) if mx else None,
+                    reasons=reasons, samples=len(self.rows))
+
+
+def dist_setup(backend):
+    import torch
+    import torch.distributed as dist
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        from datetime import timedelta
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=600))
+    return ws, rank, local
+
+
+def max_over_ranks(x: float, ws: int, device=None) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def workload_desc(layer) -> str:
+    dt = layer.w_dtype
+    if layer.n_mats > 1:
+        return (f"{layer.name}: {layer.n_mats} x W[{layer.c_out},{layer.c_in}] {dt}, "
+                f"X[{layer.n_tok},{layer.c_in}] bf16 grouped by expert")
+    return f"{layer.name}: W[{layer.c_out},{layer.c_in}] {dt}, X[{layer.n_tok},{layer.c_in}] bf16"
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+def oracle_step(layer, W_f32, n_sweep: int, rng) -> tuple[float, float, float, int]:
+    """Times the oracle on one bounded sample of the step: the full Hessian
+    (up to 4096 tokens, scaled by token count), `n_sweep` sampled blocks of
+    the sweep, and fake-quant of 8 sampled rows. Returns (estimated seconds for
+    the whole step, hessian s, sweep s, sampled blocks)."""
+    import oracle
+    n_tok = layer.n_tok
+    t_h = min(n_tok, 4096)
+    Xs = layer.X[:t_h]
+    off = None
+    if layer.offsets is not None:
+        off = np.minimum(layer.offsets, t_h)
+    t0 = time.perf_counter()
+    H = oracle.hessian(Xs, c_in=layer.c_in, offsets=off)
+    th = (time.perf_counter() - t0) * (n_tok / t_h)
+    J = layer.c_in // 16
+    amax = np.array([oracle.absmax(W_f32[m]) for m in range(layer.n_mats)], np.float32) \
+        if layer.n_mats <= 4 else np.max(np.abs(W_f32), axis=(1, 2)).astype(np.float32)
+    mats = rng.integers(0, layer.n_mats, n_sweep)
+    rows = rng.integers(0, layer.c_out, n_sweep)
+    cols = rng.integers(0, J, n_sweep)
+    Hfull = np.broadcast_to(H, (layer.n_mats,) + H.shape[1:]) if H.shape[0] == 1 else H
+    t0 = time.perf_counter()
+    codes, _, _ = oracle.sweep_blocks(W_f32, amax, np.ascontiguousarray(Hfull), mats, rows, cols)
+    ts = (time.perf_counter() - t0) * (layer.n_blocks / n_sweep)
+    nr = 8
+    t0 = time.perf_counter()
+    for i in range(nr):
+        m, r = int(mats[i]), int(rows[i])
+        oracle.fake_quant(W_f32[m, r:r + 1], amax[m:m + 1], np.ones((1, J), np.uint8))
+    tf = (time.perf_counter() - t0) * (layer.n_mats * layer.c_out / nr)
+    return th + ts + tf, th, ts, n_sweep
+
+
+def run_reference(args):
+    ws, rank, _ = dist_setup("gloo")
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    oracle.build()
+    layer = synth.make_config(args.config)
+    W_f32 = layer.W_f32()
+    rng = np.random.default_rng(0)
+    n_sweep = 4000
+    for _ in range(args.warmup):
+        oracle_step(layer, W_f32, 400, rng)
+    est = []
+    for _ in range(args.steps):
+        est.append(oracle_step(layer, W_f32, n_sweep, rng)[0])
+    t = float(sum(est))
+    value = layer.n_blocks * args.steps / t
+    sample = (f"per step: full Hessian (<=4096 tokens, scaled), {n_sweep} random blocks of the sweep, "
+              f"8 rows of fake-quant; times scaled to the whole layer")
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                ms_per_step=1e3 * t / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f64", data="synthetic", impl="reference",
+                config=dict(workload=workload_desc(layer), l2="n/a (CPU)", parallelism="none"),
+                cpu_baseline=dict(value=value, unit=UNIT, cores=1, kind="oracle", sample=sample),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0),
+                gpu_launches=0)
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- CUDA path
+def run_ours(args):
+    import torch
+    ws, rank, local = dist_setup("nccl")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import scale_calibration_b200 as lh
+    import synth
+
+    layer = synth.make_config(args.config)
+    n_mats, c_out, c_in, n_tok = layer.n_mats, layer.c_out, layer.c_in, layer.n_tok
+    J = c_in // 16
+    grouped = layer.offsets is not None
+    n_groups = n_mats if grouped else 1
+
+    if layer.w_dtype == "bf16":
+        W_host = torch.from_numpy(layer.W.view(np.int16)).view(torch.bfloat16)
+    else:
+        W_host = torch.from_numpy(np.ascontiguousarray(layer.W))
+    X_host = torch.from_numpy(layer.X.view(np.int16)).view(torch.bfloat16)
+    W = W_host.to(dev)
+    X = X_host.to(dev)
+    off = torch.from_numpy(layer.offsets).to(dev) if grouped else None
+
+    amax = torch.empty(n_mats, dtype=torch.float32, device=dev)
+    H = torch.zeros(n_groups, J, 16, 16, dtype=torch.float32, device=dev)
+    wsb = lh.lh_hessian_workspace_bytes(n_tok, c_in, n_groups)
+    wsp = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    codes = torch.empty(n_mats, c_out, J, dtype=torch.uint8, device=dev)
+    bamax = torch.empty(n_mats, c_out, J, dtype=torch.float32, device=dev)
+    Wq = torch.empty(n_mats, c_out, c_in, dtype=W.dtype, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 1 << 28) // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    ld = W.stride(1)
+    launches_per_step = 1 + 2 + (1 if grouped else 0) + 1 + 1
+
+    def step(ev=None):
+        H.zero_()
+        if ev: ev[0].record(stream)
+        lh.lh_absmax(W, W, n_mats, c_out, c_in, ld, amax, s)
+        if ev: ev[1].record(stream)
+        lh.lh_accumulate_hessian(X, lh.LH_BF16, n_tok, c_in, X.stride(0), off, n_groups, H, wsp, wsb, s)
+        if ev: ev[2].record(stream)
+        lh.lh_sweep_scales(W, W, n_mats, c_out, c_in, ld, amax, H, bamax, codes, s)
+        if ev: ev[3].record(stream)
+        lh.lh_fake_quant(W, W, n_mats, c_out, c_in, ld, amax, codes, Wq, Wq, s)
+        if ev: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    assert lh.lh_workspace_status(wsp, s) == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for i in range(args.steps):
+        flush.zero_()  # cold L2 for every step
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if ws > 1:
+        torch.distributed.barrier()
+    per = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(4)] for e in evs])  # ms [steps, 4]
+    t_rank = float(per.sum()) / 1e3
+    t_all = max_over_ranks(t_rank, ws, dev)
+    value = n_mats * c_out * J * ws * args.steps / t_all
+    t_abs, t_hess, t_sweep, t_fq = (float(x) for x in per.mean(axis=0))  # ms
+
+    # ---- end to end through the public API with host buffers
+    W_pin = W_host.pin_memory()
+    X_pin = X_host.pin_memory()
+    off_host = torch.from_numpy(layer.offsets).pin_memory() if grouped else None
+    codes_pin = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
+    bam_pin = torch.empty(bamax.shape, dtype=bamax.dtype).pin_memory()
+    Wq_pin = torch.empty(Wq.shape, dtype=Wq.dtype).pin_memory()
+
+    def e2e_step():
+        W.copy_(W_pin, non_blocking=True)
+        X.copy_(X_pin, non_blocking=True)
+        if grouped:
+            off.copy_(off_host, non_blocking=True)
+        step()
+        codes_pin.copy_(codes, non_blocking=True)
+        bam_pin.copy_(bamax, non_blocking=True)
+        Wq_pin.copy_(Wq, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        torch.distributed.barrier()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_e2e = max_over_ranks(e_start.elapsed_time(e_end) / 1e3, ws, dev)
+    h2d = W.numel() * W.element_size() + X.numel() * X.element_size() + (off.numel() * 8 if grouped else 0)
+    d2h = codes.numel() + bamax.numel() * 4 + Wq.numel() * Wq.element_size()
+    e2e = dict(value=n_mats * c_out * J * ws * args.steps / t_e2e, unit=UNIT, h2d_bytes_per_step=int(h2d),
+               d2h_bytes_per_step=int(d2h))
+
+    # ---- rooflines
+    peaks = load_peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    fp32_peak = sms * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s
+    n_blocks = n_mats * c_out * J
+    sweep_tflops = SWEEP_FLOP_PER_BLOCK * n_blocks / (t_sweep / 1e3) / 1e12
+    hess_bytes = 2 * c_in * n_tok
+    hess_gbs = hess_bytes / (t_hess / 1e3) / 1e9
+    roofline = dict(bound="alu", kernel="sweep_kernel", achieved=sweep_tflops, peak=fp32_peak, unit="TFLOP/s",
+                    frac=sweep_tflops / fp32_peak, traffic=None,
+                    peak_note=f"FP32 CUDA-core peak {sms} SMs x 128 lanes x 2 flop x {peaks['sm_max_mhz']:.0f} MHz",
+                    flop_per_block=SWEEP_FLOP_PER_BLOCK)
+    if clocks.get("sm_mhz"):
+        roofline["frac_at_measured_clock"] = sweep_tflops / (fp32_peak * clocks["sm_mhz"] / peaks["sm_max_mhz"])
+    hessian = dict(tokens_per_s=n_tok * ws / (t_hess / 1e3) if t_hess > 0 else None, bound="hbm",
+                   achieved=hess_gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=hess_gbs / peaks["hbm_gbs"],
+                   bytes_per_launch=hess_bytes, peak_source=peaks["source"])
+
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=ws, steps=args.steps, warmup=args.warmup,
+                ms_per_step=1e3 * t_all / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f32", data="synthetic",
+                config=dict(workload=workload_desc(layer), blocks=n_blocks, tokens=n_tok, l2="flushed",
+                            parallelism=f"{ws} independent layers, no collective"),
+                kernels_ms=dict(absmax=t_abs, hessian=t_hess, sweep=t_sweep, fake_quant=t_fq),
+                sweep_blocks_per_s=n_blocks * ws / (t_sweep / 1e3), roofline=roofline, hessian=hessian,
+                e2e=e2e, gpu_launches=launches_per_step * args.steps, clocks=clocks)
+
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rng = np.random.default_rng(1)
+        W_f32 = layer.W_f32()
+        t0 = time.perf_counter()
+        tot, th, tsw, ns = 0.0, 0.0, 0.0, 0
+        reps = 0
+        while time.perf_counter() - t0 < args.cpu_seconds and reps < 50:
+            e, a, b, n = oracle_step(layer, W_f32, 20000, rng)
+            tot += e; th += a; tsw += b; ns += n; reps += 1
+        cpu_value = n_blocks * reps / tot
+        line["cpu_baseline"] = dict(value=cpu_value, unit=UNIT, cores=1, kind="oracle",
+                                    sample=(f"{reps} x (full Hessian of <=4096 tokens, 20000 random sweep blocks, "
+                                            f"8 fake-quant rows), scaled to the whole layer"))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1, help="0 tiny, 1 attn_proj, 2 mlp_up, 3 mlp_down, 4 moe_experts")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,147 @@
+/*
+ * lh.h — C ABI of the Local-Hessian NVFP4 block-scale calibration library
+ * (B200, sm_100a).
+ *
+ * The method ("NVIDIA Model Optimizer Local-Hessian: 基于局部 Hessian 的 NVFP4
+ * 逐块权重缩放算法实战指南", xxmr.cn/news/266017, section "算法原理"): for a
+ * linear layer Y = W X with W [C_out, C_in] and calibration activations X
+ * (token-major here, [N tokens, C_in]), every NVFP4 block of 16 consecutive
+ * weights w_b = W[r, 16j:16j+16] gets the FP8 E4M3 block scale s that
+ * minimises the output-error proxy E_b(s) = dw^T H_j dw, where
+ * dw = Cast_E2M1(w/s)*s - w and H_j = X_j X_j^T is the 16x16 local Hessian of
+ * the block's 16 input channels. All 126 positive finite non-zero E4M3 codes
+ * (0x01..0x7E) are tried as candidates s = fp8(c) * g, g = global_amax/(6*448).
+ *
+ * Conventions (all entry points):
+ *   - Pointers marked "device" are caller-owned device memory of the current
+ *     CUDA device; the library allocates nothing (the Hessian partial sums
+ *     live in a caller-provided workspace).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call is asynchronous on that stream and returns without
+ *     synchronising; a kernel fault surfaces at the caller's next sync.
+ *   - Arguments are validated on the host before any launch. On an error
+ *     status nothing was launched and no output was touched.
+ *   - Matrices are row-major. Leading dimensions are in elements.
+ *   - bf16 and f32 element pointers must be 16-byte aligned and leading
+ *     dimensions must keep every row 16-byte aligned (LH_ERR_ALIGNMENT).
+ *   - Outputs must not alias inputs.
+ *   - Thread safety: calls are re-entrant; the only host state is a
+ *     thread-local error message.
+ */
+#ifndef LH_H_
+#define LH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LH_API __attribute__((visibility("default")))
+#else
+#define LH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LH_OK = 0,
+    LH_ERR_INVALID_ARG = 1,   /* null pointer, negative size, ld < cols, ...      */
+    LH_ERR_UNSUPPORTED = 2,   /* c_in not a multiple of 16, unknown dtype, no GPU */
+    LH_ERR_ALIGNMENT = 3,     /* pointer or row not 16-byte aligned                */
+    LH_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required        */
+    LH_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed              */
+    LH_ERR_TIMEOUT = 6        /* a bounded in-kernel wait gave up (see lh_workspace_status) */
+} lh_status;
+
+typedef enum { LH_BF16 = 0, LH_F32 = 1 } lh_dtype;
+
+/* Human-readable name of a status code (static string). */
+LH_API const char* lh_status_string(lh_status s);
+
+/* Detail of the last error returned on this host thread (e.g. the CUDA error
+ * name and which argument failed). Empty string if none. */
+LH_API const char* lh_last_error_message(void);
+
+/* ------------------------------------------------------------------------
+ * Global amax. "算法原理" (kernel contract): the sweep receives the global
+ * FP32 amax of the weight tensor. out_amax[m] = max |W_m| over the matrix
+ * [rows, cols] (leading dimension ld) of each of n_mats matrices stored back
+ * to back (matrix stride rows*ld). Exact (a max is order-independent).
+ *   W: device, bf16 or f32.  out_amax: device f32 [n_mats], overwritten.
+ * ---------------------------------------------------------------------- */
+LH_API lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t rows, int64_t cols,
+                    int64_t ld, float* out_amax, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Local Hessian accumulation. "算法原理": the local Hessian of block column j
+ * is X_j X_j^T (16x16); "入口 API 与校准流程" Phase 2: H = sum X^T X over the
+ * calibration tokens; kernel contract: H laid out [C_in/16, 16, 16].
+ *
+ *   H[g][j][a][b] += sum_{t in group g} x[t][16j+a] * x[t][16j+b]
+ *
+ * X: device bf16 [n_tokens_total, ld_x] (first c_in columns used), token-major.
+ * offsets: device int64 [n_groups+1] with the token range of each group (one
+ *   per matrix / expert: tokens [offsets[g], offsets[g+1])), or NULL for a
+ *   single group of all tokens (n_groups must then be 1). Offsets are clamped
+ *   to [0, n_tokens_total] and empty or inverted ranges count as empty.
+ * H: device f32 [n_groups][c_in/16][16][16], read and written (H += ...):
+ *   accumulation can be split over batches and resumed across calls.
+ * workspace: device, at least lh_hessian_workspace_bytes(...) bytes, 256-byte
+ *   aligned, owned by the caller; it holds per-chunk partial sums and must not
+ *   be shared by calls in flight at the same time.
+ * Numerics: bf16 products are exact in FP32; tensor-core FP32 accumulation
+ *   over at most 128 tokens, then FP64 accumulation and one final rounding.
+ * n_tokens_total == 0 is a no-op returning LH_OK.
+ * ---------------------------------------------------------------------- */
+LH_API size_t lh_hessian_workspace_bytes(int64_t n_tokens_total, int64_t c_in, int64_t n_groups);
+
+LH_API lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int64_t n_tokens_total, int64_t c_in,
+                                int64_t ld_x, const int64_t* offsets, int64_t n_groups, float* H,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Status a kernel left in `workspace` (LH_OK or LH_ERR_TIMEOUT when a bounded
+ * wait inside lh_accumulate_hessian gave up). Synchronises `stream`. */
+LH_API lh_status lh_workspace_status(const void* workspace, void* stream);
+
+/* ------------------------------------------------------------------------
+ * FP8 block-scale sweep. "算法原理": per 16-weight block, all 126 FP8 E4M3
+ * candidate scales are tried and the one minimising dw^T H dw is kept; the
+ * kernel contract takes weights as [N_BLOCKS, 16] row-major over
+ * (cout, cin/16), the global FP32 amax and H [cin/16, 16, 16], and returns
+ * the per-block best amax. For every matrix m and block (r, j):
+ *
+ *   g     = fp32(global_amax[m] / 2688)
+ *   s_c   = fp32(e4m3(c) * g),              c = 1..126
+ *   q_i   = E2M1_RNE_sat(fp32(w_i / s_c))   (q = 0 when s_c == 0)
+ *   E(c)  = dw^T H[m][j] dw,  dw = q*s_c - w
+ *   best_code[m][r][j] = argmin_c E(c)  (lowest code on ties)
+ *   best_amax[m][r][j] = fp32(6 * s_best)
+ *
+ * E is evaluated in FP32; blocks whose two best candidates are closer than a
+ * proven bound on the FP32 rounding error are re-evaluated in FP64, so the
+ * chosen code is the exact argmin up to FP64 rounding.
+ * W: device bf16 or f32 [n_mats][c_out][ld_w]. global_amax: device f32 [n_mats].
+ * H: device f32 [n_mats][c_in/16][16][16] (symmetric; the upper triangle is read).
+ * best_amax: device f32 [n_mats][c_out][c_in/16]. best_code: device u8, same shape.
+ * ---------------------------------------------------------------------- */
+LH_API lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                          int64_t ld_w, const float* global_amax, const float* H, float* best_amax,
+                          uint8_t* best_code, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Fake quantisation with the chosen codes. "算法原理": Q(W, s) = Cast(W/s)*s.
+ *   W_out[m][r][c] = cast_out( fp32( E2M1_RNE_sat(fp32(w/s)) * s ) ),
+ *   s = fp32(e4m3(codes[m][r][c/16]) * fp32(global_amax[m]/2688)).
+ * W: device [n_mats][c_out][ld_w]. codes: device u8 [n_mats][c_out][c_in/16].
+ * W_out: device [n_mats][c_out][c_in] (dense), bf16 (round to nearest even) or f32.
+ * ---------------------------------------------------------------------- */
+LH_API lh_status lh_fake_quant(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                        int64_t ld_w, const float* global_amax, const uint8_t* codes, void* W_out,
+                        lh_dtype out_dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LH_H_ */

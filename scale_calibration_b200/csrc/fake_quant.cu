@@ -1,0 +1,193 @@
+// Fake quantisation with the chosen block scales, and the global abs-max.
+//
+// "NVIDIA Model Optimizer Local-Hessian: 基于局部 Hessian 的 NVFP4 逐块权重缩放
+// 算法实战指南" (xxmr.cn/news/266017), section "算法原理": Q(W, s) = Cast(W/s) * s
+// with the per-block FP8 scale s and the global FP32 amax of the tensor.
+//
+// Both kernels stream W once from HBM: one thread per 16-weight block
+// (32 or 64 contiguous bytes, 16-byte vector loads and stores).
+#include "common.cuh"
+#include "quant.cuh"
+
+namespace lh {
+namespace {
+
+template <typename T>
+struct Vec16;
+
+template <>
+struct Vec16<uint16_t> {
+    __device__ static void load(const uint16_t* p, float (&w)[16]) {
+        const uint4* q = reinterpret_cast<const uint4*>(p);
+        const uint4 a = __ldg(q), b = __ldg(q + 1);
+        const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            w[2 * i] = __uint_as_float(v[i] << 16);
+            w[2 * i + 1] = __uint_as_float(v[i] & 0xFFFF0000u);
+        }
+    }
+    __device__ static void store(uint16_t* p, const float (&o)[16]) {
+        uint32_t v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);  // RNE
+            v[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        uint4* q = reinterpret_cast<uint4*>(p);
+        q[0] = make_uint4(v[0], v[1], v[2], v[3]);
+        q[1] = make_uint4(v[4], v[5], v[6], v[7]);
+    }
+};
+
+template <>
+struct Vec16<float> {
+    __device__ static void load(const float* p, float (&w)[16]) {
+        const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 t = __ldg(q + i);
+            w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
+        }
+    }
+    __device__ static void store(float* p, const float (&o)[16]) {
+        float4* q = reinterpret_cast<float4*>(p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    }
+};
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) fake_quant_kernel(const Tin* __restrict__ W, int64_t c_out, int64_t J,
+                                                         int64_t ld, const float* __restrict__ gamax,
+                                                         const uint8_t* __restrict__ codes,
+                                                         Tout* __restrict__ out, int64_t n_blocks_total) {
+    const int64_t per_mat = c_out * J;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks_total;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = b / per_mat;
+        const int64_t rj = b - m * per_mat;
+        const int64_t r = rj / J, j = rj - r * J;
+        const float g = __fdiv_rn(__ldg(gamax + m), 2688.0f);
+        const float s = __fmul_rn(e4m3_value(__ldg(codes + b)), g);
+        float w[16], o[16];
+        Vec16<Tin>::load(W + (m * c_out + r) * ld + 16 * j, w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float q = (s != 0.0f) ? e2m1_rne(__fdiv_rn(w[i], s)) : copysignf(0.0f, w[i]);
+            o[i] = __fmul_rn(q, s);
+        }
+        Vec16<Tout>::store(out + (m * c_out + r) * (J * 16) + 16 * j, o);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) absmax_kernel(const T* __restrict__ W, int64_t rows, int64_t cols,
+                                                     int64_t ld, unsigned int* __restrict__ out) {
+    const int64_t m = blockIdx.y;
+    const T* base = W + m * rows * ld;
+    constexpr int V = 16 / sizeof(T);  // elements per 16-byte vector
+    const int64_t nv = cols / V;
+    const int warps = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31;
+    float mx = 0.0f;
+    for (int64_t r = (int64_t)blockIdx.x * warps + (threadIdx.x >> 5); r < rows; r += (int64_t)gridDim.x * warps) {
+        const T* row = base + r * ld;
+        for (int64_t v = lane; v < nv; v += 32) {
+            const uint4 t = __ldg(reinterpret_cast<const uint4*>(row) + v);
+            const uint32_t u[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (sizeof(T) == 2) {
+                    mx = fmaxf(mx, fabsf(__uint_as_float(u[i] << 16)));
+                    mx = fmaxf(mx, fabsf(__uint_as_float(u[i] & 0xFFFF0000u)));
+                } else {
+                    mx = fmaxf(mx, fabsf(__uint_as_float(u[i])));
+                }
+            }
+        }
+        for (int64_t c = nv * V + lane; c < cols; c += 32) {
+            const float x = sizeof(T) == 2 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[c])
+                                           : reinterpret_cast<const float*>(row)[c];
+            mx = fmaxf(mx, fabsf(x));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    __shared__ float red[32];
+    if (lane == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float v = 0.0f;
+        for (int i = 0; i < warps; ++i) v = fmaxf(v, red[i]);
+        atomicMax(out + m, __float_as_uint(v));  // non-negative floats order like their bits
+    }
+}
+
+}  // namespace
+}  // namespace lh
+
+extern "C" lh_status lh_fake_quant(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                                   int64_t ld_w, const float* global_amax, const uint8_t* codes, void* W_out,
+                                   lh_dtype out_dtype, void* stream) {
+    using namespace lh;
+    clear_error();
+    if (!valid_dtype(w_dtype) || !valid_dtype(out_dtype)) return fail(LH_ERR_UNSUPPORTED, "unknown dtype");
+    if (!W || !global_amax || !codes || !W_out) return fail(LH_ERR_INVALID_ARG, "null pointer argument");
+    if (n_mats < 1 || c_out < 0 || c_in < 0) return fail(LH_ERR_INVALID_ARG, "n_mats must be >= 1, sizes >= 0");
+    if (c_in % 16 != 0) return fail(LH_ERR_UNSUPPORTED, "c_in=%lld is not a multiple of 16", (long long)c_in);
+    if (ld_w < c_in) return fail(LH_ERR_INVALID_ARG, "ld_w < c_in");
+    if (!aligned16(W) || (ld_w * elem_bytes(w_dtype)) % 16 != 0 || !aligned16(W_out))
+        return fail(LH_ERR_ALIGNMENT, "W and W_out must be 16-byte aligned with 16-byte aligned rows");
+    if (W == W_out) return fail(LH_ERR_INVALID_ARG, "W_out must not alias W");
+    const int64_t J = c_in / 16;
+    const int64_t nb = n_mats * c_out * J;
+    if (nb == 0) return LH_OK;
+    const int sms = sm_count();
+    if (sms <= 0) return fail(LH_ERR_CUDA, "no CUDA device");
+    int64_t blocks = (nb + 255) / 256;
+    if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned gb = (unsigned)blocks;
+    if (w_dtype == LH_BF16 && out_dtype == LH_BF16)
+        fake_quant_kernel<uint16_t, uint16_t><<<gb, 256, 0, st>>>((const uint16_t*)W, c_out, J, ld_w, global_amax,
+                                                                 codes, (uint16_t*)W_out, nb);
+    else if (w_dtype == LH_BF16)
+        fake_quant_kernel<uint16_t, float><<<gb, 256, 0, st>>>((const uint16_t*)W, c_out, J, ld_w, global_amax,
+                                                              codes, (float*)W_out, nb);
+    else if (out_dtype == LH_BF16)
+        fake_quant_kernel<float, uint16_t><<<gb, 256, 0, st>>>((const float*)W, c_out, J, ld_w, global_amax,
+                                                              codes, (uint16_t*)W_out, nb);
+    else
+        fake_quant_kernel<float, float><<<gb, 256, 0, st>>>((const float*)W, c_out, J, ld_w, global_amax, codes,
+                                                           (float*)W_out, nb);
+    return cuda_status(cudaGetLastError(), "fake_quant_kernel launch");
+}
+
+extern "C" lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t rows, int64_t cols,
+                               int64_t ld, float* out_amax, void* stream) {
+    using namespace lh;
+    clear_error();
+    if (!valid_dtype(w_dtype)) return fail(LH_ERR_UNSUPPORTED, "unknown dtype");
+    if (!W || !out_amax) return fail(LH_ERR_INVALID_ARG, "null pointer argument");
+    if (n_mats < 1 || rows < 0 || cols < 0 || ld < cols) return fail(LH_ERR_INVALID_ARG, "bad sizes");
+    if (n_mats > 65535) return fail(LH_ERR_UNSUPPORTED, "n_mats must be <= 65535");
+    if (!aligned16(W) || (ld * elem_bytes(w_dtype)) % 16 != 0)
+        return fail(LH_ERR_ALIGNMENT, "W must be 16-byte aligned with 16-byte aligned rows");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    lh_status s = cuda_status(cudaMemsetAsync(out_amax, 0, sizeof(float) * (size_t)n_mats, st), "memset amax");
+    if (s != LH_OK) return s;
+    if (rows == 0 || cols == 0) return LH_OK;
+    const int sms = sm_count();
+    if (sms <= 0) return fail(LH_ERR_CUDA, "no CUDA device");
+    int64_t per = (rows + 7) / 8;  // 8 warps per CTA, one row per warp per pass
+    int64_t cap = ((int64_t)sms * 8 + n_mats - 1) / n_mats;
+    if (cap < 1) cap = 1;
+    if (per > cap) per = cap;
+    dim3 grid((unsigned)per, (unsigned)n_mats);
+    if (w_dtype == LH_BF16)
+        absmax_kernel<uint16_t><<<grid, 256, 0, st>>>((const uint16_t*)W, rows, cols, ld, (unsigned int*)out_amax);
+    else
+        absmax_kernel<float><<<grid, 256, 0, st>>>((const float*)W, rows, cols, ld, (unsigned int*)out_amax);
+    return cuda_status(cudaGetLastError(), "absmax_kernel launch");
+}

@@ -1,0 +1,259 @@
+// FP8 block-scale sweep: for every NVFP4 block, all 126 E4M3 candidate
+// scales, keep the argmin of dw^T H dw.
+//
+// Method: "NVIDIA Model Optimizer Local-Hessian: 基于局部 Hessian 的 NVFP4 逐块
+// 权重缩放算法实战指南" (xxmr.cn/news/266017), section "算法原理": the
+// block-diagonal error E_b(s_b) = Delta_b (X_b X_b^T) Delta_b^T, swept over the
+// 126 FP8 candidates per block; kernel contract: weights [N_BLOCKS, 16] in
+// (cout, cin/16) order, global FP32 amax, H [cin/16, 16, 16], per-block best
+// amax out.
+//
+// Design (B200, FP32 CUDA cores):
+//  * One thread owns one block (row r, block column j); a CTA covers 128 rows
+//    of one block column, so the 16x16 H_j is staged once in shared memory
+//    and read by broadcast.
+//  * Candidate scales come in 8 mantissa classes m * 2^x (m = 1 + f/8). Within
+//    a class, consecutive codes double the scale exactly, so fp32(w / s_c) is
+//    fp32(w / s_c0) scaled by a power of two: 16 IEEE divisions per class
+//    replace 16 per candidate, and each candidate rounds the same quotient
+//    onto the E2M1 grid scaled by 2^k (exact, see e2m1_grid_round).
+//  * E(c) is evaluated in FP32 with the symmetric form (136 FMA). Its
+//    rounding error is at most ~35 u * sum|dw_a||H_ab||dw_b| (u = 2^-24), and
+//    |dw_i| <= |w_i|, so every block whose runner-up is within twice that bound
+//    of the best is re-swept in FP64 by the whole warp. The result is the
+//    exact argmin (up to FP64 rounding), lowest code on ties.
+#include "common.cuh"
+#include "quant.cuh"
+
+namespace lh {
+namespace {
+
+constexpr int kThreads = 128;  // rows per CTA
+
+// packed upper-triangle index of (a, b), a <= b
+__host__ __device__ constexpr int tri(int a, int b) { return a * 16 - (a * (a - 1)) / 2 + (b - a); }
+
+template <typename T>
+__device__ __forceinline__ void load_block(const T* p, float (&w)[16]);
+
+template <>
+__device__ __forceinline__ void load_block<uint16_t>(const uint16_t* p, float (&w)[16]) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+    const uint4 a = __ldg(q), b = __ldg(q + 1);
+    const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        w[2 * i] = __uint_as_float(v[i] << 16);
+        w[2 * i + 1] = __uint_as_float(v[i] & 0xFFFF0000u);
+    }
+}
+
+template <>
+__device__ __forceinline__ void load_block<float>(const float* p, float (&w)[16]) {
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 t = __ldg(q + i);
+        w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
+    }
+}
+
+// E4M3 code of the value (1 + f/8) * 2^x (f in 0..7, x >= -9), or the
+// subnormal code (8 + f) * 2^(x + 6) when x < -6.
+__device__ __forceinline__ int class_code(int f, int x) {
+    return x >= -6 ? 8 * (x + 7) + f : (8 + f) >> (-6 - x);
+}
+
+// FP64 error of candidate code c for block w (definition order of the method:
+// s = fp32(v(c) g), q = E2M1(fp32(w/s)), dw = q s - w exact, E = dw^T H dw).
+__device__ double candidate_error_f64(const float (&w)[16], float g, int c, const float* Hf) {
+    const float s = __fmul_rn(e4m3_value(c), g);
+    double dw[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float q = (s != 0.0f) ? e2m1_rne(__fdiv_rn(w[i], s)) : 0.0f;
+        dw[i] = (double)q * (double)s - (double)w[i];
+    }
+    double E = 0.0;
+#pragma unroll 1
+    for (int a = 0; a < 16; ++a) {
+        double t = 0.0;
+#pragma unroll
+        for (int b = 0; b < 16; ++b) t = fma((double)Hf[a * 16 + b], dw[b], t);
+        E = fma(dw[a], t, E);
+    }
+    return E;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J,
+                                                         int64_t ld, int64_t mat_stride,
+                                                         const float* __restrict__ gamax,
+                                                         const float* __restrict__ H,
+                                                         float* __restrict__ best_amax,
+                                                         uint8_t* __restrict__ best_code) {
+    __shared__ float Hf[256];
+    __shared__ float U[136];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int64_t j = blockIdx.y;
+    const int64_t m = blockIdx.z;
+    const int64_t r = (int64_t)blockIdx.x * kThreads + tid;
+    const bool active = r < c_out;
+
+    const float* Hj = H + (m * J + j) * 256;
+    for (int i = tid; i < 256; i += kThreads) Hf[i] = Hj[i];
+    __syncthreads();
+    for (int i = tid; i < 256; i += kThreads) {
+        const int a = i >> 4, b = i & 15;
+        if (a == b) U[tri(a, a)] = Hf[i];
+        else if (a < b) U[tri(a, b)] = __fadd_rn(Hf[i], Hf[b * 16 + a]);  // H_ab + H_ba
+    }
+    __syncthreads();
+
+    float w[16];
+    if (active) load_block<T>(W + m * mat_stride + r * ld + 16 * j, w);
+    else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = 0.0f;
+    }
+
+    const float A = gamax[m];
+    const float g = __fdiv_rn(A, 2688.0f);
+    // Power-of-two relation between the candidates of a class holds while
+    // every candidate scale is a normal FP32 number: g * 2^-9 >= 2^-126.
+    const bool fast = (g >= 1.2037062e-35f) && (g <= 1.0e30f);  // g >= 2^-116
+
+    float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
+    int best_c = 1;
+    bool flag = !fast;
+    if (g == 0.0f) flag = false;  // every s_c is 0: q = 0, all errors equal, code 1
+
+    if (fast) {
+        float aw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) aw[i] = fabsf(w[i]);
+        // Tw = sum |w_a| |H_ab| |w_b| bounds sum |dw_a| |H_ab| |dw_b| for every candidate.
+        float Tw = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 16; ++a) {
+            float t = fabsf(U[tri(a, a)]) * aw[a];
+#pragma unroll
+            for (int b = a + 1; b < 16; ++b) t = fmaf(fabsf(U[tri(a, b)]), aw[b], t);
+            Tw = fmaf(aw[a], t, Tw);
+        }
+
+#pragma unroll 1
+        for (int f = 0; f < 8; ++f) {
+            const int tz = (f == 0) ? 3 : (f == 4) ? 2 : (f == 2 || f == 6) ? 1 : 0;
+            const int x0 = -6 - tz;                  // smallest exponent of the class
+            const int n = (f == 7 ? 7 : 8) - x0 + 1;  // codes in the class
+            // v0 = (1 + f/8) * 2^x0, exact
+            const float v0 = (float)(8 + f) * __int_as_float((x0 - 3 + 127) << 23);
+            const float s0 = __fmul_rn(v0, g);
+            float u0[16], ss[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                u0[i] = __fdiv_rn(aw[i], s0);
+                ss[i] = copysignf(s0, w[i]);
+            }
+#pragma unroll 1
+            for (int k = 0; k < n; ++k) {
+                const int code = class_code(f, x0 + k);
+                const float lim = __int_as_float(((129 + k) << 23) | 0x400000);  // 6 * 2^k
+                const int emin = (127 + k) << 23;
+                float dw[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float q = e2m1_grid_round(u0[i], lim, emin);  // = 2^k * E2M1(u0 / 2^k)
+                    dw[i] = fmaf(q, ss[i], -w[i]);                      // q_c * s_c - w, one rounding
+                }
+                float E = 0.0f;
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    float t = U[tri(a, a)] * dw[a];
+#pragma unroll
+                    for (int b = a + 1; b < 16; ++b) t = fmaf(U[tri(a, b)], dw[b], t);
+                    E = fmaf(dw[a], t, E);
+                }
+                if (E < best_e || (E == best_e && code < best_c)) {
+                    second_e = fminf(second_e, best_e);
+                    best_e = E;
+                    best_c = code;
+                } else {
+                    second_e = fminf(second_e, E);
+                }
+            }
+        }
+        // |E32 - E| <= 35 u T <= 35 u Tw per candidate; 48 u leaves slack for
+        // the rounding of Tw itself.
+        const float kappa = 48.0f * 5.9604645e-8f;
+        const float margin = 2.0f * kappa * Tw;
+        if (!(second_e - best_e > margin)) flag = true;  // also catches NaN / inf
+    }
+
+    // FP64 re-sweep of flagged blocks, one block at a time across the warp.
+    unsigned pending = __ballot_sync(0xFFFFFFFFu, flag && active);
+    while (pending) {
+        const int src = __ffs(pending) - 1;
+        pending &= pending - 1;
+        float wv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) wv[i] = __shfl_sync(0xFFFFFFFFu, w[i], src);
+        double be = 0.0;
+        int bc = 127;
+        for (int c = lane + 1; c <= 126; c += 32) {
+            const double e = candidate_error_f64(wv, g, c, Hf);
+            if (bc == 127 || e < be) { be = e; bc = c; }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const double oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+            const int oc = __shfl_xor_sync(0xFFFFFFFFu, bc, off);
+            // lexicographic (error, code) minimum; NaN errors never win
+            const bool take = (oc != 127) && (bc == 127 || oe < be || (oe == be && oc < bc) ||
+                                              (be != be && oe == oe));
+            if (take) { be = oe; bc = oc; }
+        }
+        if (lane == src) best_c = (bc >= 1 && bc <= 126) ? bc : 1;
+    }
+
+    if (active) {
+        const int64_t o = (m * c_out + r) * J + j;
+        best_code[o] = (uint8_t)best_c;
+        best_amax[o] = __fmul_rn(6.0f, __fmul_rn(e4m3_value(best_c), g));
+    }
+}
+
+}  // namespace
+}  // namespace lh
+
+extern "C" lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out,
+                                     int64_t c_in, int64_t ld_w, const float* global_amax, const float* H,
+                                     float* best_amax, uint8_t* best_code, void* stream) {
+    using namespace lh;
+    clear_error();
+    if (!valid_dtype(w_dtype)) return fail(LH_ERR_UNSUPPORTED, "w_dtype %d is not LH_BF16 or LH_F32", (int)w_dtype);
+    if (!W || !global_amax || !H || !best_amax || !best_code)
+        return fail(LH_ERR_INVALID_ARG, "null pointer argument");
+    if (n_mats < 1 || c_out < 0 || c_in < 0) return fail(LH_ERR_INVALID_ARG, "n_mats must be >= 1, sizes >= 0");
+    if (c_in % 16 != 0) return fail(LH_ERR_UNSUPPORTED, "c_in=%lld is not a multiple of 16", (long long)c_in);
+    if (ld_w < c_in) return fail(LH_ERR_INVALID_ARG, "ld_w=%lld < c_in=%lld", (long long)ld_w, (long long)c_in);
+    if (!aligned16(W) || (ld_w * elem_bytes(w_dtype)) % 16 != 0)
+        return fail(LH_ERR_ALIGNMENT, "W must be 16-byte aligned with 16-byte aligned rows");
+    const int64_t J = c_in / 16;
+    if (J > 65535 || n_mats > 65535) return fail(LH_ERR_UNSUPPORTED, "c_in/16 and n_mats must be <= 65535");
+    if (c_out == 0 || J == 0) return LH_OK;
+    const int64_t tiles = (c_out + kThreads - 1) / kThreads;
+    if (tiles > 0x7FFFFFFF) return fail(LH_ERR_UNSUPPORTED, "c_out too large");
+    dim3 grid((unsigned)tiles, (unsigned)J, (unsigned)n_mats);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t mat_stride = c_out * ld_w;
+    if (w_dtype == LH_BF16)
+        sweep_kernel<uint16_t><<<grid, kThreads, 0, st>>>(static_cast<const uint16_t*>(W), c_out, J, ld_w,
+                                                          mat_stride, global_amax, H, best_amax, best_code);
+    else
+        sweep_kernel<float><<<grid, kThreads, 0, st>>>(static_cast<const float*>(W), c_out, J, ld_w, mat_stride,
+                                                       global_amax, H, best_amax, best_code);
+    return cuda_status(cudaGetLastError(), "sweep_kernel launch");
+}

@@ -1,0 +1,102 @@
+"""The C ABI on the host: the library loads without a GPU, exports every
+symbol include/lh.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lh():
+    import scale_calibration_b200 as lh
+    return lh
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "lh.h")).read()
+    return sorted(set(re.findall(r"LH_API\s+[\w\s\*]*?\b(lh_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    lh = _lh()
+    names = declared_functions()
+    assert len(names) >= 8
+    lib = ctypes.CDLL(lh._binding.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(lh.EXPORTS) == names
+
+
+def test_status_strings():
+    lh = _lh()
+    assert lh.lh_status_string(0) == "LH_OK"
+    assert lh.lh_status_string(6) == "LH_ERR_TIMEOUT"
+    assert lh.lh_status_string(99) == "LH_ERR_UNKNOWN"
+
+
+FAKE = 0x10000000  # a 256-byte-aligned address that is never dereferenced: validation fails first
+
+
+def test_sweep_rejects_bad_arguments():
+    lh = _lh()
+    ok = dict(W=FAKE, w_dtype=lh.LH_BF16, n_mats=1, c_out=64, c_in=128, ld_w=128, global_amax=FAKE, H=FAKE,
+              best_amax=FAKE, best_code=FAKE, stream=0, check=False)
+    cases = [
+        (dict(W=0), 1), (dict(H=0), 1), (dict(best_code=0), 1), (dict(n_mats=0), 1), (dict(c_out=-1), 1),
+        (dict(c_in=24, ld_w=24), 2), (dict(ld_w=120), 1), (dict(W=FAKE + 2), 3), (dict(ld_w=132), 3),
+        (dict(w_dtype=7), 2), (dict(c_in=16 * 70000, ld_w=16 * 70000), 2),
+    ]
+    for over, want in cases:
+        a = dict(ok, **over)
+        assert lh.lh_sweep_scales(**a) == want, over
+        assert lh.lh_last_error_message() != ""
+
+
+def test_sweep_empty_is_noop():
+    lh = _lh()
+    assert lh.lh_sweep_scales(FAKE, lh.LH_BF16, 1, 0, 128, 128, FAKE, FAKE, FAKE, FAKE, 0, check=False) == 0
+
+
+def test_hessian_rejects_bad_arguments():
+    lh = _lh()
+    need = lh.lh_hessian_workspace_bytes(300, 64, 1)
+    ok = dict(X=FAKE, x_dtype=lh.LH_BF16, n_tokens_total=300, c_in=64, ld_x=64, offsets=None, n_groups=1, H=FAKE,
+              workspace=FAKE, workspace_bytes=need, stream=0, check=False)
+    cases = [
+        (dict(x_dtype=lh.LH_F32), 2), (dict(X=0), 1), (dict(H=0), 1), (dict(n_groups=2), 1),
+        (dict(c_in=40, ld_x=40), 2), (dict(ld_x=60), 1), (dict(ld_x=68), 3), (dict(X=FAKE + 8), 3),
+        (dict(workspace_bytes=need - 1), 4), (dict(workspace=0), 4), (dict(workspace=FAKE + 16), 3),
+        (dict(n_tokens_total=-1), 1), (dict(n_groups=0), 1),
+    ]
+    for over, want in cases:
+        a = dict(ok, **over)
+        assert lh.lh_accumulate_hessian(**a) == want, over
+
+
+def test_hessian_zero_tokens_is_noop():
+    lh = _lh()
+    assert lh.lh_accumulate_hessian(FAKE, lh.LH_BF16, 0, 64, 64, None, 1, FAKE, 0, 0, 0, check=False) == 0
+
+
+def test_workspace_size_grows_with_tokens_and_groups():
+    lh = _lh()
+    a = lh.lh_hessian_workspace_bytes(2048, 4096, 1)
+    b = lh.lh_hessian_workspace_bytes(16384, 4096, 1)
+    c = lh.lh_hessian_workspace_bytes(2048, 4096, 64)
+    J = 4096 // 16
+    assert a >= 256 + J * 1024 and b >= a and c > a
+    assert lh.lh_hessian_workspace_bytes(100, 0, 1) == 0
+
+
+def test_fake_quant_and_absmax_reject_bad_arguments():
+    lh = _lh()
+    ok = dict(W=FAKE, w_dtype=lh.LH_BF16, n_mats=1, c_out=8, c_in=32, ld_w=32, global_amax=FAKE, codes=FAKE,
+              W_out=FAKE + 4096, out_dtype=lh.LH_BF16, stream=0, check=False)
+    for over, want in [(dict(W_out=FAKE), 1), (dict(codes=0), 1), (dict(c_in=20, ld_w=20), 2),
+                       (dict(out_dtype=3), 2), (dict(W_out=FAKE + 4100), 3)]:
+        assert lh.lh_fake_quant(**dict(ok, **over)) == want, over
+    assert lh.lh_absmax(FAKE, lh.LH_F32, 1, 4, 8, 4, FAKE, 0, check=False) == 1
+    assert lh.lh_absmax(0, lh.LH_F32, 1, 4, 8, 8, FAKE, 0, check=False) == 1
+    assert lh.lh_absmax(FAKE + 4, lh.LH_F32, 1, 4, 8, 8, FAKE, 0, check=False) == 3
