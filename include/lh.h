@@ -105,6 +105,29 @@ LH_API lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int64_t 
 LH_API lh_status lh_workspace_status(const void* workspace, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Allocation-free variant of lh_accumulate_hessian. The pages have no
+ * counterpart: this is a library convenience for callers that cannot
+ * allocate device memory when they calibrate (serving processes that reserve
+ * nearly all HBM for their own pools at start-up, plugins whose host owns
+ * every device allocation, callers that avoid cudaMalloc/cudaFree because
+ * those can synchronise the device). Same arguments and result as
+ * lh_accumulate_hessian minus the workspace, which comes from a fixed 16 MiB
+ * array compiled into the library; every GPU that loads the library holds it
+ * until the process exits. Calls no cudaMalloc/cudaFree.
+ *   - Returns LH_ERR_WORKSPACE, without launching, when
+ *     lh_hessian_workspace_bytes(n_tokens_total, c_in, n_groups) > 16 MiB.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the array (it keeps the last call's contents; what must
+ *     start at zero is cleared by each call). Calls whose kernels overlap on
+ *     the GPU race on it: serialise them (one stream, one thread at a time).
+ * ---------------------------------------------------------------------- */
+LH_API lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, int64_t n_tokens_total,
+                                               int64_t c_in, int64_t ld_x, const int64_t* offsets,
+                                               int64_t n_groups, float* H, void* stream);
+
+/* ------------------------------------------------------------------------
  * FP8 block-scale sweep. "算法原理": per 16-weight block, all 126 FP8 E4M3
  * candidate scales are tried and the one minimising dw^T H dw is kept; the
  * kernel contract takes weights as [N_BLOCKS, 16] row-major over

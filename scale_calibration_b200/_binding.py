@@ -19,6 +19,7 @@ LH_BF16, LH_F32 = 0, 1
 EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
+    "lh_accumulate_hessian_noalloc",
 ]
 
 
@@ -40,6 +41,7 @@ def _load() -> ctypes.CDLL:
         "lh_hessian_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64]),
         "lh_accumulate_hessian": (I32, [P, I32, I64, I64, I64, P, I64, P, P, ctypes.c_size_t, P]),
         "lh_workspace_status": (I32, [P, P]),
+        "lh_accumulate_hessian_noalloc": (I32, [P, I32, I64, I64, I64, P, I64, P, P]),
         "lh_sweep_scales": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P]),
         "lh_fake_quant": (I32, [P, I32, I64, I64, I64, I64, P, P, P, I32, P]),
     }
@@ -115,6 +117,17 @@ def lh_accumulate_hessian(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_gro
                                    _ptr(H), _ptr(workspace), workspace_bytes, _stream(stream))
     if check:
         _check(s, "lh_accumulate_hessian")
+    return s
+
+
+def lh_accumulate_hessian_noalloc(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H, stream=None,
+                                  check=True) -> int:
+    """lh_accumulate_hessian with the workspace taken from the library's own
+    fixed 16 MiB device array, for callers that cannot allocate device memory."""
+    s = _lib.lh_accumulate_hessian_noalloc(_ptr(X), _dtype(x_dtype), n_tokens_total, c_in, ld_x, _ptr(offsets),
+                                           n_groups, _ptr(H), _stream(stream))
+    if check:
+        _check(s, "lh_accumulate_hessian_noalloc")
     return s
 
 

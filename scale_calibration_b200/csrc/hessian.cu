@@ -569,3 +569,66 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
         kp.partial, offsets ? kfirst : nullptr, J, plain_chunks, H);
     return cuda_status(cudaGetLastError(), "hessian_reduce_kernel launch");
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of lh_accumulate_hessian.
+//
+// Some callers cannot allocate device memory when they calibrate: serving
+// processes that reserve nearly all HBM for their own pools at start-up,
+// plugins whose host owns every device allocation and offers them no
+// allocator, and latency-sensitive callers that avoid cudaMalloc/cudaFree
+// because those calls can synchronise the whole device. This entry point
+// takes the Hessian workspace from a fixed array compiled into the library
+// instead of from the caller. Every GPU that loads the library holds the
+// array (kNoAllocScratchBytes) until the process exits.
+//
+// In host code `lh_noalloc_scratch` names a host-side stand-in, not a device
+// address; its device address is looked up once per device with
+// cudaGetSymbolAddress on the first call made with that device current, and
+// that lookup is the only set-up. Make the first call on each device before
+// any stream capture. All calls share the one array: the header words that
+// must start at zero are cleared by every call, and calls whose kernels
+// overlap on the GPU (different streams, or different host threads) race on
+// the array and must be serialised by the caller.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;  // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char lh_noalloc_scratch[kNoAllocScratchBytes];
+
+extern "C" lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, int64_t n_tokens_total,
+                                                   int64_t c_in, int64_t ld_x, const int64_t* offsets,
+                                                   int64_t n_groups, float* H, void* stream) {
+    using namespace lh;
+    clear_error();
+    const size_t need = lh_hessian_workspace_bytes(n_tokens_total, c_in, n_groups);
+    if (n_tokens_total == 0 || c_in == 0 || need == 0)  // no-op or invalid sizes: the checks of the main entry
+        return lh_accumulate_hessian(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H, nullptr, 0,
+                                     stream);
+    if (need > kNoAllocScratchBytes)
+        return fail(LH_ERR_WORKSPACE,
+                    "this Hessian needs %zu bytes of scratch but the allocation-free entry point has %zu "
+                    "(16 MiB); call lh_accumulate_hessian with a caller-provided workspace instead",
+                    need, kNoAllocScratchBytes);
+    int dev = 0;
+    lh_status s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+    if (s != LH_OK) return s;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(LH_ERR_UNSUPPORTED, "device index %d too large", dev);
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* p = nullptr;
+            s = cuda_status(cudaGetSymbolAddress(&p, lh_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+            if (s != LH_OK) return s;
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    return lh_accumulate_hessian(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H, scratch,
+                                 kNoAllocScratchBytes, stream);
+}

@@ -1,0 +1,57 @@
+"""The allocation-free Hessian entry point against the workspace one (needs a B200).
+
+lh_accumulate_hessian_noalloc serves callers that cannot allocate device
+memory when they calibrate (processes whose HBM is already reserved by their
+own pools, plugins whose host owns every allocation, callers avoiding the
+device-wide synchronisation of cudaMalloc/cudaFree). It must give the same H
+as lh_accumulate_hessian with a caller workspace, call after call, although
+every call reuses the library's one fixed scratch array. This file sorts last
+so that a run stopping at the first failure has run every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from scale_calibration_b200._binding import LH_ERR_WORKSPACE
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+def _hessians(layer):
+    import scale_calibration_b200 as lh
+    _, X, off = gu.to_device(layer)
+    n_groups = layer.n_mats if off is not None else 1
+    J = layer.c_in // 16
+    H_ws = torch.zeros(n_groups, J, 16, 16, dtype=torch.float32, device="cuda")
+    wsb = lh.lh_hessian_workspace_bytes(layer.n_tok, layer.c_in, n_groups)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    lh.lh_accumulate_hessian(X, lh.LH_BF16, layer.n_tok, layer.c_in, X.stride(0), off, n_groups, H_ws, ws, wsb)
+    H_na = torch.zeros_like(H_ws)
+    lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, layer.n_tok, layer.c_in, X.stride(0), off, n_groups, H_na)
+    torch.cuda.synchronize()
+    return H_ws.cpu().numpy(), H_na.cpu().numpy()
+
+
+def test_noalloc_matches_workspace_entry_on_consecutive_calls(cuda_ok):
+    layers = [
+        synth.make_layer(8, 128, 2552, seed=21, n_mats=8, counts=[0, 5, 1, 300, 0, 17, 129, 2100]),
+        synth.make_layer(4, 4096, 2048, seed=22),      # attention-projection-sized X
+    ]
+    for layer in layers:   # two calls in a row, different shapes, on the shared scratch array
+        H_ws, H_na = _hessians(layer)
+        per, whole, bad = gu.hessian_rel_errors(H_na, H_ws.astype(np.float64))
+        assert per <= gu.HESSIAN_RTOL and whole <= gu.HESSIAN_RTOL and bad == 0, (per, whole, bad)
+        assert np.array_equal(H_ws, H_na)  # same kernels, deterministic order
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
+    import scale_calibration_b200 as lh
+    n_tok, c_in = 65536, 32768   # needs far more than 16 MiB of partial sums
+    assert lh.lh_hessian_workspace_bytes(n_tok, c_in, 1) > (16 << 20)
+    H = torch.zeros(1, dtype=torch.float32, device="cuda")
+    X = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    s = lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, n_tok, c_in, c_in, None, 1, H, check=False)
+    assert s == LH_ERR_WORKSPACE
+    assert "16 MiB" in lh.lh_last_error_message()
