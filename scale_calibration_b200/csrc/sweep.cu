@@ -25,10 +25,15 @@
 #include "common.cuh"
 #include "quant.cuh"
 
+#ifndef LH_SWEEP_UREGS
+#define LH_SWEEP_UREGS false  // form coefficients read from shared memory (more warps per SM)
+#endif
+
 namespace lh {
 namespace {
 
-constexpr int kThreads = 128;  // rows per CTA
+constexpr int kThreads = 128;        // threads per CTA (one block per thread at a time)
+constexpr int kRowsPerThread = 4;    // rows each thread walks; a CTA covers 512 rows of one block column
 
 // packed upper-triangle index of (a, b), a <= b
 __host__ __device__ constexpr int tri(int a, int b) { return a * 16 - (a * (a - 1)) / 2 + (b - a); }
@@ -85,38 +90,118 @@ __device__ double candidate_error_f64(const float (&w)[16], float g, int c, cons
     return E;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J,
-                                                         int64_t ld, int64_t mat_stride,
-                                                         const float* __restrict__ gamax,
-                                                         const float* __restrict__ H,
-                                                         float* __restrict__ best_amax,
-                                                         uint8_t* __restrict__ best_code) {
-    __shared__ float Hf[256];
-    __shared__ float U[136];
+// Pair (U[a][2i], U[a][2i+1]) of row a of the symmetric form, in the order
+// the form consumes them: rows a = 0..15, for row a the column pairs
+// i = ceil(a/2)..7 (for even a the first pair starts on the diagonal; for odd
+// a the diagonal is kept apart in Ud[a/2]). Every row's run of pairs starts
+// on a 16-byte boundary so two pairs come in one 128-bit shared load.
+__host__ __device__ constexpr int pair_first(int a) { return (a + 1) / 2; }
+__host__ __device__ constexpr int pair_count(int a) { return 8 - pair_first(a); }
+__host__ __device__ constexpr int pair_offset(int a) {
+    int o = 0;
+    for (int r = 0; r < a; ++r) o += 2 * ((pair_count(r) + 1) / 2);
+    return o;
+}
+constexpr int kPairSlots = pair_offset(16);
+static_assert(kPairSlots == 72, "72 padded pair slots");
+
+struct SweepShared {
+    float2 Up[kPairSlots];  // U pairs (U_ab = H_aa on the diagonal, H_ab + H_ba above it)
+    float Ud[8];            // diagonals of the odd rows
+    float Ua[136];          // |U| packed upper triangle, for the error bound
+    float Hf[256];          // H as given, for the FP64 re-sweep
+};
+
+__device__ __forceinline__ float4 lds128(const void* p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+    return v;
+}
+
+// E = sum_{a<=b} U_ab dw_a dw_b with packed FP32 FMAs: for every row a the
+// pair (t.x, t.y) accumulates the even and odd columns b >= a, then
+// E += dw_a (t.x + t.y). 64 paired FMAs, 8 products, 16 adds, 16 FMAs.
+// Coefficients from registers.
+__device__ __forceinline__ float quad_form_regs(const float2 (&dw)[8], const float2 (&Up)[kPairSlots],
+                                                const float (&Ud)[8]) {
+    float E = 0.0f;
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+        const float dwa = (a & 1) ? dw[a >> 1].y : dw[a >> 1].x;
+        float2 t = (a & 1) ? make_float2(Ud[a >> 1] * dwa, 0.0f) : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = pair_first(a); i < 8; ++i) t = __ffma2_rn(Up[pair_offset(a) + i - pair_first(a)], dw[i], t);
+        E = fmaf(dwa, t.x + t.y, E);
+    }
+    return E;
+}
+
+// The same form with the coefficients streamed from shared memory on every
+// call (volatile 128-bit broadcast loads: the compiler may not keep them).
+__device__ __forceinline__ float quad_form_smem(const float2 (&dw)[8], const SweepShared& sm) {
+    const float4 d0 = lds128(&sm.Ud[0]), d1 = lds128(&sm.Ud[4]);
+    const float ud[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    float E = 0.0f;
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+        const float dwa = (a & 1) ? dw[a >> 1].y : dw[a >> 1].x;
+        float2 t = (a & 1) ? make_float2(ud[a >> 1] * dwa, 0.0f) : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = pair_first(a); i < 8; i += 2) {
+            const float4 c = lds128(&sm.Up[pair_offset(a) + i - pair_first(a)]);
+            t = __ffma2_rn(make_float2(c.x, c.y), dw[i], t);
+            if (i + 1 < 8) t = __ffma2_rn(make_float2(c.z, c.w), dw[i + 1], t);
+        }
+        E = fmaf(dwa, t.x + t.y, E);
+    }
+    return E;
+}
+
+template <typename T, bool kURegs>
+__global__ void __launch_bounds__(kThreads, kURegs ? 2 : 3)
+sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int64_t mat_stride,
+             const float* __restrict__ gamax, const float* __restrict__ H, float* __restrict__ best_amax,
+             uint8_t* __restrict__ best_code) {
+    __shared__ __align__(16) SweepShared sm;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int64_t j = blockIdx.y;
     const int64_t m = blockIdx.z;
-    const int64_t r = (int64_t)blockIdx.x * kThreads + tid;
-    const bool active = r < c_out;
 
     const float* Hj = H + (m * J + j) * 256;
-    for (int i = tid; i < 256; i += kThreads) Hf[i] = Hj[i];
+    for (int i = tid; i < 256; i += kThreads) sm.Hf[i] = Hj[i];
+    for (int i = tid; i < kPairSlots; i += kThreads) sm.Up[i] = make_float2(0.0f, 0.0f);
     __syncthreads();
     for (int i = tid; i < 256; i += kThreads) {
         const int a = i >> 4, b = i & 15;
-        if (a == b) U[tri(a, a)] = Hf[i];
-        else if (a < b) U[tri(a, b)] = __fadd_rn(Hf[i], Hf[b * 16 + a]);  // H_ab + H_ba
+        if (b < a) continue;
+        const float u = (a == b) ? sm.Hf[i] : __fadd_rn(sm.Hf[i], sm.Hf[b * 16 + a]);  // H_ab + H_ba
+        sm.Ua[tri(a, b)] = fabsf(u);
+        if ((a & 1) && b == a) {
+            sm.Ud[a >> 1] = u;  // odd rows keep their diagonal apart
+        } else {
+            // column b sits in pair b/2 of row a, as .x (even b) or .y (odd b)
+            float* dst = reinterpret_cast<float*>(&sm.Up[pair_offset(a) + (b >> 1) - pair_first(a)]);
+            dst[b & 1] = u;
+        }
     }
     __syncthreads();
 
-    float w[16];
-    if (active) load_block<T>(W + m * mat_stride + r * ld + 16 * j, w);
-    else {
+    // form coefficients: copied into registers, or read from shared memory (broadcast)
+    float2 Ur[kPairSlots];
+    float Udr[8];
+    if constexpr (kURegs) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = 0.0f;
+        for (int i = 0; i < kPairSlots; ++i) Ur[i] = sm.Up[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) Udr[i] = sm.Ud[i];
     }
+    auto form = [&](const float2 (&d)[8]) -> float {
+        if constexpr (kURegs) return quad_form_regs(d, Ur, Udr);
+        else return quad_form_smem(d, sm);
+    };
 
     const float A = gamax[m];
     const float g = __fdiv_rn(A, 2688.0f);
@@ -124,104 +209,125 @@ __global__ void __launch_bounds__(kThreads) sweep_kernel(const T* __restrict__ W
     // every candidate scale is a normal FP32 number: g * 2^-9 >= 2^-126.
     const bool fast = (g >= 1.2037062e-35f) && (g <= 1.0e30f);  // g >= 2^-116
 
-    float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
-    int best_c = 1;
-    bool flag = !fast;
-    if (g == 0.0f) flag = false;  // every s_c is 0: q = 0, all errors equal, code 1
-
-    if (fast) {
-        float aw[16];
+#pragma unroll 1
+    for (int rr = 0; rr < kRowsPerThread; ++rr) {
+        const int64_t r = ((int64_t)blockIdx.x * kRowsPerThread + rr) * kThreads + tid;
+        const bool active = r < c_out;
+        if (__all_sync(0xFFFFFFFFu, !active)) break;
+        float w[16];
+        if (active) load_block<T>(W + m * mat_stride + r * ld + 16 * j, w);
+        else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) aw[i] = fabsf(w[i]);
-        // Tw = sum |w_a| |H_ab| |w_b| bounds sum |dw_a| |H_ab| |dw_b| for every candidate.
-        float Tw = 0.0f;
-#pragma unroll
-        for (int a = 0; a < 16; ++a) {
-            float t = fabsf(U[tri(a, a)]) * aw[a];
-#pragma unroll
-            for (int b = a + 1; b < 16; ++b) t = fmaf(fabsf(U[tri(a, b)]), aw[b], t);
-            Tw = fmaf(aw[a], t, Tw);
+            for (int i = 0; i < 16; ++i) w[i] = 0.0f;
         }
+
+        float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
+        int best_c = 1;
+        bool flag = !fast;
+        if (g == 0.0f) flag = false;  // every s_c is 0: q = 0, all errors equal, code 1
+
+        if (fast) {
+            // Tw = sum_{a<=b} |U_ab| |w_a| |w_b| bounds sum |U_ab| |dw_a| |dw_b| for every candidate.
+            float Tw = 0.0f;
+#pragma unroll
+            for (int a = 0; a < 16; ++a) {
+                float t = sm.Ua[tri(a, a)] * fabsf(w[a]);
+#pragma unroll
+                for (int b = a + 1; b < 16; ++b) t = fmaf(sm.Ua[tri(a, b)], fabsf(w[b]), t);
+                Tw = fmaf(fabsf(w[a]), t, Tw);
+            }
+            float2 nw[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) nw[p] = make_float2(-w[2 * p], -w[2 * p + 1]);
 
 #pragma unroll 1
-        for (int f = 0; f < 8; ++f) {
-            const int tz = (f == 0) ? 3 : (f == 4) ? 2 : (f == 2 || f == 6) ? 1 : 0;
-            const int x0 = -6 - tz;                  // smallest exponent of the class
-            const int n = (f == 7 ? 7 : 8) - x0 + 1;  // codes in the class
-            // v0 = (1 + f/8) * 2^x0, exact
-            const float v0 = (float)(8 + f) * __int_as_float((x0 - 3 + 127) << 23);
-            const float s0 = __fmul_rn(v0, g);
-            float u0[16], ss[16];
+            for (int f = 0; f < 8; ++f) {
+                const int tz = (f == 0) ? 3 : (f == 4) ? 2 : (f == 2 || f == 6) ? 1 : 0;
+                const int x0 = -6 - tz;                  // smallest exponent of the class
+                const int n = (f == 7 ? 7 : 8) - x0 + 1;  // codes in the class
+                const float v0 = (float)(8 + f) * __int_as_float((x0 - 3 + 127) << 23);  // (1 + f/8) 2^x0
+                const float s0 = __fmul_rn(v0, g);
+                float2 u[8], ss[8];
+                unsigned ep[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                u0[i] = __fdiv_rn(aw[i], s0);
-                ss[i] = copysignf(s0, w[i]);
-            }
+                for (int p = 0; p < 8; ++p) {
+                    const float u0 = __fdiv_rn(fabsf(w[2 * p]), s0);
+                    const float u1 = __fdiv_rn(fabsf(w[2 * p + 1]), s0);
+                    u[p] = make_float2(u0, u1);
+                    ss[p] = make_float2(copysignf(s0, w[2 * p]), copysignf(s0, w[2 * p + 1]));
+                    ep[2 * p] = (__float_as_uint(u0) & 0x7F800000u) + 0x0B400000u;
+                    ep[2 * p + 1] = (__float_as_uint(u1) & 0x7F800000u) + 0x0B400000u;
+                }
 #pragma unroll 1
-            for (int k = 0; k < n; ++k) {
-                const int code = class_code(f, x0 + k);
-                const float lim = __int_as_float(((129 + k) << 23) | 0x400000);  // 6 * 2^k
-                const int emin = (127 + k) << 23;
-                float dw[16];
+                for (int k = 0; k < n; ++k) {
+                    const int code = class_code(f, x0 + k);
+                    const float lim = __int_as_float(((129 + k) << 23) | 0x400000);  // 6 * 2^k
+                    const unsigned mlo = ((unsigned)(127 + k) << 23) + 0x0B400000u;
+                    const unsigned mhi = ((unsigned)(129 + k) << 23) + 0x0B400000u;
+                    float2 dw[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float q = e2m1_grid_round(u0[i], lim, emin);  // = 2^k * E2M1(u0 / 2^k)
-                    dw[i] = fmaf(q, ss[i], -w[i]);                      // q_c * s_c - w, one rounding
-                }
-                float E = 0.0f;
-#pragma unroll
-                for (int a = 0; a < 16; ++a) {
-                    float t = U[tri(a, a)] * dw[a];
-#pragma unroll
-                    for (int b = a + 1; b < 16; ++b) t = fmaf(U[tri(a, b)], dw[b], t);
-                    E = fmaf(dw[a], t, E);
-                }
-                if (E < best_e || (E == best_e && code < best_c)) {
-                    second_e = fminf(second_e, best_e);
-                    best_e = E;
-                    best_c = code;
-                } else {
-                    second_e = fminf(second_e, E);
+                    for (int p = 0; p < 8; ++p) {
+                        // q = min(RNE of u on the grid 2^k {0,.5,1,1.5,2,3,4,6,...}, 6 * 2^k): the
+                        // magic constant M = 1.5 * 2^23 * spacing comes from the binade of u
+                        // clamped to [2^k, 4 * 2^k]; (u + M) - M rounds u to the spacing with
+                        // ties to even, and values past 6 * 2^k land at or above it.
+                        const float2 M = make_float2(__uint_as_float(min(max(ep[2 * p], mlo), mhi)),
+                                                     __uint_as_float(min(max(ep[2 * p + 1], mlo), mhi)));
+                        const float2 t = __fadd2_rn(u[p], M);
+                        float2 q = __ffma2_rn(M, make_float2(-1.0f, -1.0f), t);  // t - M, exact
+                        q.x = fminf(q.x, lim);
+                        q.y = fminf(q.y, lim);
+                        dw[p] = __ffma2_rn(q, ss[p], nw[p]);  // q_c s_c - w, one rounding
+                    }
+                    const float E = form(dw);
+                    if (E < best_e) {
+                        second_e = best_e;
+                        best_e = E;
+                        best_c = code;
+                    } else {
+                        second_e = fminf(second_e, E);
+                    }
                 }
             }
+            // |E32 - E| <= 30 u T <= 30 u Tw per candidate (u = 2^-24); 48 u leaves slack
+            // for the rounding of Tw itself. Exact FP32 ties (second == best) are flagged
+            // too, so the FP64 re-sweep applies the lowest-code rule.
+            const float kappa = 48.0f * 5.9604645e-8f;
+            const float margin = 2.0f * kappa * Tw;
+            if (!(second_e - best_e > margin)) flag = true;  // also catches NaN / inf
         }
-        // |E32 - E| <= 35 u T <= 35 u Tw per candidate; 48 u leaves slack for
-        // the rounding of Tw itself.
-        const float kappa = 48.0f * 5.9604645e-8f;
-        const float margin = 2.0f * kappa * Tw;
-        if (!(second_e - best_e > margin)) flag = true;  // also catches NaN / inf
-    }
 
-    // FP64 re-sweep of flagged blocks, one block at a time across the warp.
-    unsigned pending = __ballot_sync(0xFFFFFFFFu, flag && active);
-    while (pending) {
-        const int src = __ffs(pending) - 1;
-        pending &= pending - 1;
-        float wv[16];
+        // FP64 re-sweep of flagged blocks, one block at a time across the warp.
+        unsigned pending = __ballot_sync(0xFFFFFFFFu, flag && active);
+        while (pending) {
+            const int src = __ffs(pending) - 1;
+            pending &= pending - 1;
+            float wv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) wv[i] = __shfl_sync(0xFFFFFFFFu, w[i], src);
-        double be = 0.0;
-        int bc = 127;
-        for (int c = lane + 1; c <= 126; c += 32) {
-            const double e = candidate_error_f64(wv, g, c, Hf);
-            if (bc == 127 || e < be) { be = e; bc = c; }
-        }
+            for (int i = 0; i < 16; ++i) wv[i] = __shfl_sync(0xFFFFFFFFu, w[i], src);
+            double be = 0.0;
+            int bc = 127;
+            for (int c = lane + 1; c <= 126; c += 32) {
+                const double e = candidate_error_f64(wv, g, c, sm.Hf);
+                if (bc == 127 || e < be) { be = e; bc = c; }
+            }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const double oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
-            const int oc = __shfl_xor_sync(0xFFFFFFFFu, bc, off);
-            // lexicographic (error, code) minimum; NaN errors never win
-            const bool take = (oc != 127) && (bc == 127 || oe < be || (oe == be && oc < bc) ||
-                                              (be != be && oe == oe));
-            if (take) { be = oe; bc = oc; }
+            for (int off = 16; off > 0; off >>= 1) {
+                const double oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+                const int oc = __shfl_xor_sync(0xFFFFFFFFu, bc, off);
+                // lexicographic (error, code) minimum; NaN errors never win
+                const bool take = (oc != 127) && (bc == 127 || oe < be || (oe == be && oc < bc) ||
+                                                  (be != be && oe == oe));
+                if (take) { be = oe; bc = oc; }
+            }
+            if (lane == src) best_c = (bc >= 1 && bc <= 126) ? bc : 1;
         }
-        if (lane == src) best_c = (bc >= 1 && bc <= 126) ? bc : 1;
-    }
 
-    if (active) {
-        const int64_t o = (m * c_out + r) * J + j;
-        best_code[o] = (uint8_t)best_c;
-        best_amax[o] = __fmul_rn(6.0f, __fmul_rn(e4m3_value(best_c), g));
+        if (active) {
+            const int64_t o = (m * c_out + r) * J + j;
+            best_code[o] = (uint8_t)best_c;
+            best_amax[o] = __fmul_rn(6.0f, __fmul_rn(e4m3_value(best_c), g));
+        }
     }
 }
 
@@ -244,16 +350,17 @@ extern "C" lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_
     const int64_t J = c_in / 16;
     if (J > 65535 || n_mats > 65535) return fail(LH_ERR_UNSUPPORTED, "c_in/16 and n_mats must be <= 65535");
     if (c_out == 0 || J == 0) return LH_OK;
-    const int64_t tiles = (c_out + kThreads - 1) / kThreads;
+    const int64_t rows_per_cta = (int64_t)kThreads * kRowsPerThread;
+    const int64_t tiles = (c_out + rows_per_cta - 1) / rows_per_cta;
     if (tiles > 0x7FFFFFFF) return fail(LH_ERR_UNSUPPORTED, "c_out too large");
     dim3 grid((unsigned)tiles, (unsigned)J, (unsigned)n_mats);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t mat_stride = c_out * ld_w;
     if (w_dtype == LH_BF16)
-        sweep_kernel<uint16_t><<<grid, kThreads, 0, st>>>(static_cast<const uint16_t*>(W), c_out, J, ld_w,
+        sweep_kernel<uint16_t, LH_SWEEP_UREGS><<<grid, kThreads, 0, st>>>(static_cast<const uint16_t*>(W), c_out, J, ld_w,
                                                           mat_stride, global_amax, H, best_amax, best_code);
     else
-        sweep_kernel<float><<<grid, kThreads, 0, st>>>(static_cast<const float*>(W), c_out, J, ld_w, mat_stride,
+        sweep_kernel<float, LH_SWEEP_UREGS><<<grid, kThreads, 0, st>>>(static_cast<const float*>(W), c_out, J, ld_w, mat_stride,
                                                        global_amax, H, best_amax, best_code);
     return cuda_status(cudaGetLastError(), "sweep_kernel launch");
 }
