@@ -69,6 +69,20 @@ __device__ __forceinline__ int class_code(int f, int x) {
     return x >= -6 ? 8 * (x + 7) + f : (8 + f) >> (-6 - x);
 }
 
+// Correctly rounded FP32 quotient a / b for positive normal b, from y = RN(1/b)
+// (correctly rounded reciprocal): q = RN(a y) is within one ulp of a/b, the
+// remainder a - b q is exact with one FMA, and RN(q + r y) is RN(a/b)
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990, Theorem 1; see also
+// Muller et al., Handbook of Floating-Point Arithmetic, ch. 4). Valid while
+// the remainder a - b q cannot underflow, i.e. for a >= 2^-100 (or a = 0)
+// and a normal b; blocks with a smaller non-zero |w| use IEEE division.
+__device__ __forceinline__ float div_by_recip(float a, float b, float y) {
+    const float q = __fmul_rn(a, y);
+    const float r = __fmaf_rn(-q, b, a);
+    return __fmaf_rn(r, y, q);
+}
+
 // FP64 error of candidate code c for block w (definition order of the method:
 // s = fp32(v(c) g), q = E2M1(fp32(w/s)), dw = q s - w exact, E = dw^T H dw).
 __device__ double candidate_error_f64(const float (&w)[16], float g, int c, const float* Hf) {
@@ -105,7 +119,11 @@ __host__ __device__ constexpr int pair_offset(int a) {
 constexpr int kPairSlots = pair_offset(16);
 static_assert(kPairSlots == 72, "72 padded pair slots");
 
+constexpr int kTileRows = kThreads * kRowsPerThread;  // rows of one CTA, walked in sorted order
+
 struct SweepShared {
+    unsigned long long key[kTileRows];  // (bits of min non-zero |w|) << 32 | local row, sorted
+    double Us[136];                     // H_aa, H_ab + H_ba (a < b) in FP64, packed upper triangle
     float2 Up[kPairSlots];  // U pairs (U_ab = H_aa on the diagonal, H_ab + H_ba above it)
     float Ud[8];            // diagonals of the odd rows
     float Ua[136];          // |U| packed upper triangle, for the error bound
@@ -126,16 +144,17 @@ __device__ __forceinline__ float4 lds128(const void* p) {
 // Coefficients from registers.
 __device__ __forceinline__ float quad_form_regs(const float2 (&dw)[8], const float2 (&Up)[kPairSlots],
                                                 const float (&Ud)[8]) {
-    float E = 0.0f;
+    float E0 = 0.0f, E1 = 0.0f;  // even and odd rows: two independent chains
 #pragma unroll
     for (int a = 0; a < 16; ++a) {
         const float dwa = (a & 1) ? dw[a >> 1].y : dw[a >> 1].x;
         float2 t = (a & 1) ? make_float2(Ud[a >> 1] * dwa, 0.0f) : make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int i = pair_first(a); i < 8; ++i) t = __ffma2_rn(Up[pair_offset(a) + i - pair_first(a)], dw[i], t);
-        E = fmaf(dwa, t.x + t.y, E);
+        if (a & 1) E1 = fmaf(dwa, t.x + t.y, E1);
+        else E0 = fmaf(dwa, t.x + t.y, E0);
     }
-    return E;
+    return E0 + E1;
 }
 
 // The same form with the coefficients streamed from shared memory on every
@@ -143,7 +162,7 @@ __device__ __forceinline__ float quad_form_regs(const float2 (&dw)[8], const flo
 __device__ __forceinline__ float quad_form_smem(const float2 (&dw)[8], const SweepShared& sm) {
     const float4 d0 = lds128(&sm.Ud[0]), d1 = lds128(&sm.Ud[4]);
     const float ud[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-    float E = 0.0f;
+    float E0 = 0.0f, E1 = 0.0f;  // even and odd rows: two independent chains
 #pragma unroll
     for (int a = 0; a < 16; ++a) {
         const float dwa = (a & 1) ? dw[a >> 1].y : dw[a >> 1].x;
@@ -154,9 +173,10 @@ __device__ __forceinline__ float quad_form_smem(const float2 (&dw)[8], const Swe
             t = __ffma2_rn(make_float2(c.x, c.y), dw[i], t);
             if (i + 1 < 8) t = __ffma2_rn(make_float2(c.z, c.w), dw[i + 1], t);
         }
-        E = fmaf(dwa, t.x + t.y, E);
+        if (a & 1) E1 = fmaf(dwa, t.x + t.y, E1);
+        else E0 = fmaf(dwa, t.x + t.y, E0);
     }
-    return E;
+    return E0 + E1;
 }
 
 template <typename T, bool kURegs>
@@ -179,6 +199,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         if (b < a) continue;
         const float u = (a == b) ? sm.Hf[i] : __fadd_rn(sm.Hf[i], sm.Hf[b * 16 + a]);  // H_ab + H_ba
         sm.Ua[tri(a, b)] = fabsf(u);
+        sm.Us[tri(a, b)] = (a == b) ? (double)sm.Hf[i] : (double)sm.Hf[i] + (double)sm.Hf[b * 16 + a];  // exact
         if ((a & 1) && b == a) {
             sm.Ud[a >> 1] = u;  // odd rows keep their diagonal apart
         } else {
@@ -188,6 +209,37 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         }
     }
     __syncthreads();
+
+    // Rows are walked in the order of their smallest non-zero |w|: a candidate
+    // saturates every weight of a block exactly when that minimum exceeds 5 s_c,
+    // so after sorting the 32 rows of a warp mostly agree on which candidates
+    // saturate (closed form) and the warp skips the full form together.
+    const int64_t tile0 = (int64_t)blockIdx.x * kTileRows;
+    for (int p = tid; p < kTileRows; p += kThreads) {
+        const int64_t r = tile0 + p;
+        uint32_t key = 0xFFFFFFFFu;  // rows past c_out go last
+        if (r < c_out) {
+            float wk[16];
+            load_block<T>(W + m * mat_stride + r * ld + 16 * j, wk);
+            float mn = __int_as_float(0x7F800000);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mn = (wk[i] != 0.0f) ? fminf(mn, fabsf(wk[i])) : mn;
+            key = __float_as_uint(mn);
+        }
+        sm.key[p] = ((unsigned long long)key << 32) | (unsigned)p;
+    }
+    __syncthreads();
+    for (int k2 = 2; k2 <= kTileRows; k2 <<= 1)  // bitonic sort, ascending
+        for (int jj = k2 >> 1; jj > 0; jj >>= 1) {
+            for (int i = tid; i < kTileRows; i += kThreads) {
+                const int ixj = i ^ jj;
+                if (ixj > i) {
+                    const unsigned long long x = sm.key[i], y = sm.key[ixj];
+                    if ((x > y) == ((i & k2) == 0)) { sm.key[i] = y; sm.key[ixj] = x; }
+                }
+            }
+            __syncthreads();
+        }
 
     // form coefficients: copied into registers, or read from shared memory (broadcast)
     float2 Ur[kPairSlots];
@@ -211,7 +263,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 
 #pragma unroll 1
     for (int rr = 0; rr < kRowsPerThread; ++rr) {
-        const int64_t r = ((int64_t)blockIdx.x * kRowsPerThread + rr) * kThreads + tid;
+        const int64_t r = tile0 + (int64_t)(sm.key[rr * kThreads + tid] & 0xFFFFFFFFu);
         const bool active = r < c_out;
         if (__all_sync(0xFFFFFFFFu, !active)) break;
         float w[16];
@@ -236,9 +288,37 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 for (int b = a + 1; b < 16; ++b) t = fmaf(sm.Ua[tri(a, b)], fabsf(w[b]), t);
                 Tw = fmaf(fabsf(w[a]), t, Tw);
             }
-            float2 nw[8];
+            float2 w2[8];
 #pragma unroll
-            for (int p = 0; p < 8; ++p) nw[p] = make_float2(-w[2 * p], -w[2 * p + 1]);
+            for (int p = 0; p < 8; ++p) w2[p] = make_float2(w[2 * p], w[2 * p + 1]);
+            // Closed forms in FP64 with sigma = sign(w) (0 where w = 0): a saturated
+            // candidate has dw = 6 s_c sigma - w, so E = 36 s^2 sHs - 6 s (sHw + wHs) + wHw;
+            // an all-zero candidate has dw = -w, so E = wHw.
+            double sHs = 0.0, sHw_wHs = 0.0, wHw = 0.0;
+            {
+                double wd[16], sd[16];
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    wd[a] = (double)w[a];
+                    sd[a] = (w[a] > 0.0f) ? 1.0 : (w[a] < 0.0f ? -1.0 : 0.0);
+                }
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    double tw = 0.0, ts = 0.0;  // sum_{b >= a} Us_ab w_b, Us_ab sigma_b
+#pragma unroll
+                    for (int b = a; b < 16; ++b) {
+                        const double h = sm.Us[tri(a, b)];
+                        tw = fma(h, wd[b], tw);
+                        ts = fma(h, sd[b], ts);
+                    }
+                    wHw = fma(wd[a], tw, wHw);
+                    sHs = fma(sd[a], ts, sHs);
+                    sHw_wHs = fma(sd[a], tw, fma(wd[a], ts, sHw_wHs));
+                }
+            }
+            const float E_zero = (float)wHw;
+            // the reciprocal-based quotient needs every non-zero |w| >= 2^-100
+            const bool tiny_w = __uint_as_float((uint32_t)(sm.key[rr * kThreads + tid] >> 32)) < 7.888609e-31f;
 
 #pragma unroll 1
             for (int f = 0; f < 8; ++f) {
@@ -249,14 +329,21 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 const float s0 = __fmul_rn(v0, g);
                 float2 u[8], ss[8];
                 unsigned ep[16];
+                float umin = __int_as_float(0x7F800000), umax = 0.0f;  // over the non-zero weights
+                const float rs0 = __frcp_rn(s0);
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {
-                    const float u0 = __fdiv_rn(fabsf(w[2 * p]), s0);
-                    const float u1 = __fdiv_rn(fabsf(w[2 * p + 1]), s0);
+                    const float u0 = tiny_w ? __fdiv_rn(fabsf(w[2 * p]), s0) : div_by_recip(fabsf(w[2 * p]), s0, rs0);
+                    const float u1 = tiny_w ? __fdiv_rn(fabsf(w[2 * p + 1]), s0)
+                                            : div_by_recip(fabsf(w[2 * p + 1]), s0, rs0);
                     u[p] = make_float2(u0, u1);
-                    ss[p] = make_float2(copysignf(s0, w[2 * p]), copysignf(s0, w[2 * p + 1]));
+                    // -sign(w) s0: the form is even in dw, so w - q s (= -dw) is used
+                    ss[p] = make_float2(copysignf(s0, -w[2 * p]), copysignf(s0, -w[2 * p + 1]));
                     ep[2 * p] = (__float_as_uint(u0) & 0x7F800000u) + 0x0B400000u;
                     ep[2 * p + 1] = (__float_as_uint(u1) & 0x7F800000u) + 0x0B400000u;
+                    umin = (w[2 * p] != 0.0f) ? fminf(umin, u0) : umin;
+                    umin = (w[2 * p + 1] != 0.0f) ? fminf(umin, u1) : umin;
+                    umax = fmaxf(umax, fmaxf(u0, u1));
                 }
 #pragma unroll 1
                 for (int k = 0; k < n; ++k) {
@@ -264,6 +351,17 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     const float lim = __int_as_float(((129 + k) << 23) | 0x400000);  // 6 * 2^k
                     const unsigned mlo = ((unsigned)(127 + k) << 23) + 0x0B400000u;
                     const unsigned mhi = ((unsigned)(129 + k) << 23) + 0x0B400000u;
+                    // every non-zero weight saturates (q = +-6) iff min u > 5 * 2^k; every q is 0
+                    // iff max u <= 2^k / 4 (ties 5 -> 4 and 1/4 -> 0 round to even)
+                    const bool sat = umin > __int_as_float(((129 + k) << 23) | 0x200000);  // 5 * 2^k
+                    const bool zero = umax <= __int_as_float((125 + k) << 23);              // 2^k / 4
+                    float E;
+                    if (__all_sync(0xFFFFFFFFu, sat)) {
+                        const double sc = (double)s0 * (double)__int_as_float((127 + k) << 23);  // s_c, exact
+                        E = (float)fma(fma(36.0 * sHs, sc, -6.0 * sHw_wHs), sc, wHw);
+                    } else if (__all_sync(0xFFFFFFFFu, zero)) {
+                        E = E_zero;
+                    } else {
                     float2 dw[8];
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
@@ -277,9 +375,10 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         float2 q = __ffma2_rn(M, make_float2(-1.0f, -1.0f), t);  // t - M, exact
                         q.x = fminf(q.x, lim);
                         q.y = fminf(q.y, lim);
-                        dw[p] = __ffma2_rn(q, ss[p], nw[p]);  // q_c s_c - w, one rounding
+                        dw[p] = __ffma2_rn(q, ss[p], w2[p]);  // w - q_c s_c = -dw, one rounding
                     }
-                    const float E = form(dw);
+                    E = form(dw);
+                    }
                     if (E < best_e) {
                         second_e = best_e;
                         best_e = E;

@@ -204,3 +204,15 @@ def test_mlp_down_full_size(cuda_ok):
 @pytest.mark.slow
 def test_moe_experts_full_size(cuda_ok):
     _sampled_parity(4, h_cols=24)
+
+
+def test_tiny_weights_inside_normal_blocks(cuda_ok):
+    # weights far below the global scale (down to 1e-37) next to normal ones: the
+    # quotients w/s stay exact where the sweep divides by a reciprocal and
+    # fall back to IEEE division for blocks holding such tiny values
+    layer = synth.make_layer(256, 64, 300, seed=14, w_dtype="f32")
+    rng = np.random.default_rng(14)
+    W = layer.W
+    idx = rng.choice(W.size, size=W.size // 8, replace=False)
+    W.reshape(-1)[idx] *= np.float32(10.0) ** rng.integers(-36, -2, size=idx.size).astype(np.float32)
+    _full_parity(layer)
