@@ -104,6 +104,18 @@ LH_API lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int64_t 
  * wait inside lh_accumulate_hessian gave up). Synchronises `stream`. */
 LH_API lh_status lh_workspace_status(const void* workspace, void* stream);
 
+/* Diagnostics; the pages have no counterpart. Runs on `stream` the bounded
+ * wait that the Hessian kernel uses for its mbarriers, on a barrier that
+ * nothing arrives on (arrive == 0) or that is completed first (arrive != 0),
+ * with a limit of timeout_us microseconds (1 .. 1e6). A wait that runs out
+ * records LH_ERR_TIMEOUT in the workspace header exactly as
+ * lh_accumulate_hessian does, so lh_workspace_status(workspace) then returns
+ * LH_ERR_TIMEOUT (LH_OK when arrive != 0). Lets callers exercise their
+ * handling of an expired wait without a GPU fault; the context stays usable.
+ * workspace: device, >= 256 bytes, 256-byte aligned. */
+LH_API lh_status lh_debug_wait_timeout(void* workspace, size_t workspace_bytes, int64_t timeout_us, int arrive,
+                                       void* stream);
+
 /* ------------------------------------------------------------------------
  * Allocation-free variant of lh_accumulate_hessian. The pages have no
  * counterpart: this is a library convenience for callers that cannot

@@ -19,7 +19,7 @@ LH_BF16, LH_F32 = 0, 1
 EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
-    "lh_accumulate_hessian_noalloc",
+    "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout",
 ]
 
 
@@ -42,6 +42,7 @@ def _load() -> ctypes.CDLL:
         "lh_accumulate_hessian": (I32, [P, I32, I64, I64, I64, P, I64, P, P, ctypes.c_size_t, P]),
         "lh_workspace_status": (I32, [P, P]),
         "lh_accumulate_hessian_noalloc": (I32, [P, I32, I64, I64, I64, P, I64, P, P]),
+        "lh_debug_wait_timeout": (I32, [P, ctypes.c_size_t, I64, I32, P]),
         "lh_sweep_scales": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P]),
         "lh_fake_quant": (I32, [P, I32, I64, I64, I64, I64, P, P, P, I32, P]),
     }
@@ -128,6 +129,13 @@ def lh_accumulate_hessian_noalloc(X, x_dtype, n_tokens_total, c_in, ld_x, offset
                                            n_groups, _ptr(H), _stream(stream))
     if check:
         _check(s, "lh_accumulate_hessian_noalloc")
+    return s
+
+
+def lh_debug_wait_timeout(workspace, workspace_bytes, timeout_us, arrive, stream=None, check=True) -> int:
+    s = _lib.lh_debug_wait_timeout(_ptr(workspace), workspace_bytes, timeout_us, arrive, _stream(stream))
+    if check:
+        _check(s, "lh_debug_wait_timeout")
     return s
 
 

@@ -329,6 +329,24 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(const __grid_co
     }
 }
 
+// Diagnostics: the bounded wait of the kernels above, on an mbarrier that
+// nothing arrives on (arrive == 0) or that thread 0 completes first
+// (arrive != 0); a wait that runs out records LH_ERR_TIMEOUT in the workspace
+// header like hessian_tc_kernel does.
+__global__ void wait_timeout_kernel(int* err, uint64_t timeout_ns, int arrive) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (arrive && threadIdx.x == 0) mbar_arrive(smem_u32(&bar));
+    const bool ok = mbar_wait(smem_u32(&bar), 0u, &abort_flag, timeout_ns);
+    if (!ok) atomicExch(err, (int)LH_ERR_TIMEOUT);
+}
+
 // Builds the chunk table of the grouped case: each group's token range split
 // into chunks of `chunk` tokens; kfirst[g] = first chunk of group g.
 __global__ void chunk_table_kernel(const int64_t* __restrict__ offsets, int64_t G, int64_t n_tok, int64_t chunk,
@@ -429,6 +447,21 @@ extern "C" lh_status lh_workspace_status(const void* workspace, void* stream) {
     if (s != LH_OK) return s;
     if (err != 0) return fail((lh_status)err, "a bounded wait in the Hessian kernel expired");
     return LH_OK;
+}
+
+extern "C" lh_status lh_debug_wait_timeout(void* workspace, size_t workspace_bytes, int64_t timeout_us,
+                                           int arrive, void* stream) {
+    using namespace lh;
+    clear_error();
+    if (!workspace || workspace_bytes < kHeaderBytes) return fail(LH_ERR_WORKSPACE, "workspace of 256 bytes needed");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(LH_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+    if (timeout_us < 1 || timeout_us > 1000000) return fail(LH_ERR_INVALID_ARG, "timeout_us must be in [1, 1e6]");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    lh_status s = cuda_status(cudaMemsetAsync(workspace, 0, kHeaderBytes, st), "clear workspace header");
+    if (s != LH_OK) return s;
+    wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<int*>(workspace), (uint64_t)timeout_us * 1000ull, arrive);
+    return cuda_status(cudaGetLastError(), "wait_timeout_kernel launch");
 }
 
 extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int64_t n_tokens_total, int64_t c_in,

@@ -40,16 +40,17 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Waits for the phase of `parity` to complete; false on timeout (kTimeoutNs)
-// or when *abort_flag becomes non-zero.
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// Waits for the phase of `parity` to complete; false on timeout (timeout_ns,
+// 1 s by default) or when *abort_flag becomes non-zero.
+static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              uint64_t timeout_ns = kTimeoutNs) {
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try(bar, parity)) return true;
         if ((it & 63) == 0) {
             if (*abort_flag) return false;
-            if (global_ns() - t0 > kTimeoutNs) return false;
+            if (global_ns() - t0 > timeout_ns) return false;
         }
     }
 }

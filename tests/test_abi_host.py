@@ -100,3 +100,12 @@ def test_fake_quant_and_absmax_reject_bad_arguments():
     assert lh.lh_absmax(FAKE, lh.LH_F32, 1, 4, 8, 4, FAKE, 0, check=False) == 1
     assert lh.lh_absmax(0, lh.LH_F32, 1, 4, 8, 8, FAKE, 0, check=False) == 1
     assert lh.lh_absmax(FAKE + 4, lh.LH_F32, 1, 4, 8, 8, FAKE, 0, check=False) == 3
+
+
+def test_debug_wait_rejects_bad_arguments():
+    lh = _lh()
+    assert lh.lh_debug_wait_timeout(FAKE, 255, 1000, 0, 0, check=False) == 4
+    assert lh.lh_debug_wait_timeout(0, 256, 1000, 0, 0, check=False) == 4
+    assert lh.lh_debug_wait_timeout(FAKE + 16, 256, 1000, 0, 0, check=False) == 3
+    assert lh.lh_debug_wait_timeout(FAKE, 256, 0, 0, 0, check=False) == 1
+    assert lh.lh_debug_wait_timeout(FAKE, 256, 2000000, 0, 0, check=False) == 1
