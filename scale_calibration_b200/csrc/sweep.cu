@@ -121,14 +121,57 @@ static_assert(kPairSlots == 72, "72 padded pair slots");
 
 constexpr int kTileRows = kThreads * kRowsPerThread;  // rows of one CTA, walked in sorted order
 
+constexpr int kSortBuckets = 512;
+
 struct SweepShared {
-    unsigned long long key[kTileRows];  // (bits of min non-zero |w|) << 32 | local row, sorted
+    unsigned long long key[kTileRows];    // (bits of min non-zero |w|) << 32 | local row
+    unsigned long long order[kTileRows];  // the same, grouped by sort bucket
+    uint32_t hist[kSortBuckets];
     double Us[136];                     // H_aa, H_ab + H_ba (a < b) in FP64, packed upper triangle
     float2 Up[kPairSlots];  // U pairs (U_ab = H_aa on the diagonal, H_ab + H_ba above it)
     float Ud[8];            // diagonals of the odd rows
     float Ua[136];          // |U| packed upper triangle, for the error bound
     float Hf[256];          // H as given, for the FP64 re-sweep
+    float2 dg[8];           // diagonal of H, pairs (for the lower bound)
+    float Cw[4][16][17];    // Cholesky work arrays, one per warp
+    float lcolw[4][16];
+    int pd[8];              // results of the shifted positive-definiteness tests
+    float mu;               // mu <= lambda_min(D^-1/2 H D^-1/2), D = diag(H); 0 disables pruning
 };
+
+// Is C - mu I positive definite, C = D^-1/2 H_s D^-1/2 (H_s = (H + H^T)/2,
+// rows with H_aa = 0 replaced by identity rows)? FP32 Cholesky by one warp
+// (lane i owns row i) on its own copy `Cw`; true when every pivot is positive.
+__device__ bool shifted_pd(const float* Hf, float (*Cw)[17], float* lcol, float mu, int lane) {
+    const int i = lane;
+    const bool own = i < 16;
+    if (own) {
+        const float hii = Hf[i * 17];
+        for (int b = 0; b < 16; ++b) {
+            const float hbb = Hf[b * 17];
+            float c;
+            if (hii > 0.0f && hbb > 0.0f)
+                c = (0.5f * (Hf[i * 16 + b] + Hf[b * 16 + i])) * (rsqrtf(hii) * rsqrtf(hbb));
+            else
+                c = (i == b) ? 1.0f : 0.0f;
+            Cw[i][b] = c - ((i == b) ? mu : 0.0f);
+        }
+    }
+    __syncwarp();
+    bool ok = true;
+    for (int k = 0; k < 16; ++k) {
+        const float d = Cw[k][k];
+        ok = ok && (d > 0.0f);
+        const float rl = d > 0.0f ? rsqrtf(d) : 1.0f;
+        const float l_ik = (own && i > k) ? Cw[i][k] * rl : 0.0f;
+        if (own) lcol[i] = l_ik;
+        __syncwarp();
+        if (own && i > k)
+            for (int b = k + 1; b <= i; ++b) Cw[i][b] -= l_ik * lcol[b];
+        __syncwarp();
+    }
+    return ok;
+}
 
 __device__ __forceinline__ float4 lds128(const void* p) {
     float4 v;
@@ -187,6 +230,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
     __shared__ __align__(16) SweepShared sm;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
+    const int warp = tid >> 5;
     const int64_t j = blockIdx.y;
     const int64_t m = blockIdx.z;
 
@@ -208,16 +252,57 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             dst[b & 1] = u;
         }
     }
-    __syncthreads();
+    // mu for the candidate lower bound E >= mu sum_a H_aa dw_a^2: the largest of
+    // eight shifts (two rounds, one shift per warp) at which C - mu I passes an
+    // FP32 Cholesky test. A completed factorisation is backward stable
+    // (|dC| <= 17 u |L||L^T| <= 17 u entrywise, so lambda_min(C) >= mu - 16 * 17 u);
+    // 2^-14 is subtracted to cover it. mu = 0 (no pruning) when H has a zero
+    // diagonal entry with a non-zero off-diagonal entry in its row or a negative
+    // diagonal entry, or when no shift passes.
+    {
+        bool psd_rows = true;
+        if (lane < 16) {
+            const float hii = sm.Hf[lane * 17];
+            if (!(hii >= 0.0f)) psd_rows = false;
+            if (hii == 0.0f)
+                for (int b = 0; b < 16; ++b)
+                    if (sm.Hf[lane * 16 + b] != 0.0f || sm.Hf[b * 16 + lane] != 0.0f) psd_rows = false;
+        }
+        psd_rows = __all_sync(0xFFFFFFFFu, psd_rows);
+        const float mu1 = 0.2f * (float)(warp + 1) - 0.1f;           // 0.1 0.3 0.5 0.7
+        const bool ok1 = psd_rows && shifted_pd(sm.Hf, sm.Cw[warp], sm.lcolw[warp], mu1, lane);
+        if (lane == 0) sm.pd[warp] = ok1;
+        if (tid < 8) sm.dg[tid] = make_float2(sm.Hf[(2 * tid) * 17], sm.Hf[(2 * tid + 1) * 17]);
+        __syncthreads();
+        float base = 0.0f;
+        for (int q = 0; q < 4; ++q)
+            if (sm.pd[q]) base = 0.2f * (float)(q + 1) - 0.1f;
+        const bool any1 = sm.pd[0] != 0;
+        const float mu2 = base + 0.05f * (float)(warp + 1);          // refine above the best shift
+        const bool ok2 = any1 && shifted_pd(sm.Hf, sm.Cw[warp], sm.lcolw[warp], mu2, lane);
+        if (lane == 0) sm.pd[4 + warp] = ok2;
+        __syncthreads();
+        float best = any1 ? base : 0.0f;
+        for (int q = 0; q < 4; ++q)
+            if (sm.pd[4 + q]) best = fmaxf(best, base + 0.05f * (float)(q + 1));
+        if (tid == 0) sm.mu = best > 0.0f ? best - 6.1035156e-5f : 0.0f;  // - 2^-14
+    }
 
     // Rows are walked in the order of their smallest non-zero |w|: a candidate
     // saturates every weight of a block exactly when that minimum exceeds 5 s_c,
     // so after sorting the 32 rows of a warp mostly agree on which candidates
     // saturate (closed form) and the warp skips the full form together.
     const int64_t tile0 = (int64_t)blockIdx.x * kTileRows;
-    for (int p = tid; p < kTileRows; p += kThreads) {
+    // counting sort of the tile's rows by a 9-bit key (exponent and first
+    // mantissa bit of the smallest non-zero |w|; rows past c_out last)
+    for (int i = tid; i < kSortBuckets; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    uint32_t kb[kRowsPerThread];
+#pragma unroll
+    for (int q = 0; q < kRowsPerThread; ++q) {
+        const int p = q * kThreads + tid;
         const int64_t r = tile0 + p;
-        uint32_t key = 0xFFFFFFFFu;  // rows past c_out go last
+        uint32_t key = 0xFFFFFFFFu;
         if (r < c_out) {
             float wk[16];
             load_block<T>(W + m * mat_stride + r * ld + 16 * j, wk);
@@ -226,20 +311,32 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             for (int i = 0; i < 16; ++i) mn = (wk[i] != 0.0f) ? fminf(mn, fabsf(wk[i])) : mn;
             key = __float_as_uint(mn);
         }
+        kb[q] = (key == 0xFFFFFFFFu) ? (uint32_t)(kSortBuckets - 1) : min(key >> 22, (uint32_t)(kSortBuckets - 2));
         sm.key[p] = ((unsigned long long)key << 32) | (unsigned)p;
+        atomicAdd(&sm.hist[kb[q]], 1u);
     }
     __syncthreads();
-    for (int k2 = 2; k2 <= kTileRows; k2 <<= 1)  // bitonic sort, ascending
-        for (int jj = k2 >> 1; jj > 0; jj >>= 1) {
-            for (int i = tid; i < kTileRows; i += kThreads) {
-                const int ixj = i ^ jj;
-                if (ixj > i) {
-                    const unsigned long long x = sm.key[i], y = sm.key[ixj];
-                    if ((x > y) == ((i & k2) == 0)) { sm.key[i] = y; sm.key[ixj] = x; }
-                }
-            }
-            __syncthreads();
+    if (tid < 32) {  // exclusive scan of the histogram by one warp
+        uint32_t v[kSortBuckets / 32], run = 0;
+#pragma unroll
+        for (int i = 0; i < kSortBuckets / 32; ++i) { v[i] = sm.hist[tid * (kSortBuckets / 32) + i]; run += v[i]; }
+        uint32_t incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (tid >= off) incl += o;
         }
+        uint32_t pos = incl - run;
+#pragma unroll
+        for (int i = 0; i < kSortBuckets / 32; ++i) { sm.hist[tid * (kSortBuckets / 32) + i] = pos; pos += v[i]; }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < kRowsPerThread; ++q) {
+        const uint32_t pos = atomicAdd(&sm.hist[kb[q]], 1u);
+        sm.order[pos] = sm.key[q * kThreads + tid];
+    }
+    __syncthreads();
 
     // form coefficients: copied into registers, or read from shared memory (broadcast)
     float2 Ur[kPairSlots];
@@ -263,7 +360,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 
 #pragma unroll 1
     for (int rr = 0; rr < kRowsPerThread; ++rr) {
-        const int64_t r = tile0 + (int64_t)(sm.key[rr * kThreads + tid] & 0xFFFFFFFFu);
+        const int64_t r = tile0 + (int64_t)(sm.order[rr * kThreads + tid] & 0xFFFFFFFFu);
         const bool active = r < c_out;
         if (__all_sync(0xFFFFFFFFu, !active)) break;
         float w[16];
@@ -291,6 +388,11 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             float2 w2[8];
 #pragma unroll
             for (int p = 0; p < 8; ++p) w2[p] = make_float2(w[2 * p], w[2 * p + 1]);
+            // |E32 - E| <= 30 u T <= 30 u Tw per candidate (u = 2^-24); 48 u leaves slack
+            // for the rounding of Tw itself.
+            const float margin = 2.0f * (48.0f * 5.9604645e-8f) * Tw;
+            // mu rounded down, less 32 u for the rounding of dw and of the bound's sum
+            const float mu_lb = sm.mu * (1.0f - 32.0f * 5.9604645e-8f);
             // Closed forms in FP64 with sigma = sign(w) (0 where w = 0): a saturated
             // candidate has dw = 6 s_c sigma - w, so E = 36 s^2 sHs - 6 s (sHw + wHs) + wHw;
             // an all-zero candidate has dw = -w, so E = wHw.
@@ -318,7 +420,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             }
             const float E_zero = (float)wHw;
             // the reciprocal-based quotient needs every non-zero |w| >= 2^-100
-            const bool tiny_w = __uint_as_float((uint32_t)(sm.key[rr * kThreads + tid] >> 32)) < 7.888609e-31f;
+            const bool tiny_w = __uint_as_float((uint32_t)(sm.order[rr * kThreads + tid] >> 32)) < 7.888609e-31f;
 
 #pragma unroll 1
             for (int f = 0; f < 8; ++f) {
@@ -377,7 +479,19 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         q.y = fminf(q.y, lim);
                         dw[p] = __ffma2_rn(q, ss[p], w2[p]);  // w - q_c s_c = -dw, one rounding
                     }
-                    E = form(dw);
+                    // E >= mu sum_a H_aa dw_a^2: skip the form when, for every lane, that bound
+                    // (rounded down) exceeds the best so far by more than the FP32 error margin,
+                    // so the candidate can neither be the argmin nor tie it
+                    float2 lb2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                    for (int p = 0; p < 8; p += 2) {
+                        const float4 d4 = lds128(&sm.dg[p]);
+                        lb2 = __ffma2_rn(__fmul2_rn(dw[p], dw[p]), make_float2(d4.x, d4.y), lb2);
+                        lb2 = __ffma2_rn(__fmul2_rn(dw[p + 1], dw[p + 1]), make_float2(d4.z, d4.w), lb2);
+                    }
+                    const float LB = (lb2.x + lb2.y) * mu_lb;
+                    if (__all_sync(0xFFFFFFFFu, LB > best_e + margin)) E = __int_as_float(0x7F800000);
+                    else E = form(dw);
                     }
                     if (E < best_e) {
                         second_e = best_e;
@@ -388,11 +502,8 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     }
                 }
             }
-            // |E32 - E| <= 30 u T <= 30 u Tw per candidate (u = 2^-24); 48 u leaves slack
-            // for the rounding of Tw itself. Exact FP32 ties (second == best) are flagged
-            // too, so the FP64 re-sweep applies the lowest-code rule.
-            const float kappa = 48.0f * 5.9604645e-8f;
-            const float margin = 2.0f * kappa * Tw;
+            // Exact FP32 ties (second == best) are flagged too, so the FP64 re-sweep applies
+            // the lowest-code rule.
             if (!(second_e - best_e > margin)) flag = true;  // also catches NaN / inf
         }
 
