@@ -447,8 +447,13 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     umin = (w[2 * p + 1] != 0.0f) ? fminf(umin, u1) : umin;
                     umax = fmaxf(umax, fmaxf(u0, u1));
                 }
-#pragma unroll 1
-                for (int k = 0; k < n; ++k) {
+                // One candidate; returns true when every lane proves that the rest of this
+                // pass is prunable. Pass 0 walks k upwards: the weights quantised to zero
+                // (dw_i = w_i exactly) only grow in number, so mu * sum_{q_i = 0} H_ii w_i^2
+                // bounds every later candidate. Pass 1 walks k downwards: saturated weights
+                // stay saturated and their |dw_i| = | |w_i| - 6 s_c | only grows as s_c
+                // halves, so mu * sum_{saturated} H_ii dw_i^2 bounds every later candidate.
+                auto candidate = [&](int k, bool up) -> bool {
                     const int code = class_code(f, x0 + k);
                     const float lim = __int_as_float(((129 + k) << 23) | 0x400000);  // 6 * 2^k
                     const unsigned mlo = ((unsigned)(127 + k) << 23) + 0x0B400000u;
@@ -458,40 +463,62 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     const bool sat = umin > __int_as_float(((129 + k) << 23) | 0x200000);  // 5 * 2^k
                     const bool zero = umax <= __int_as_float((125 + k) << 23);              // 2^k / 4
                     float E;
+                    bool stop = false;
                     if (__all_sync(0xFFFFFFFFu, sat)) {
                         const double sc = (double)s0 * (double)__int_as_float((127 + k) << 23);  // s_c, exact
                         E = (float)fma(fma(36.0 * sHs, sc, -6.0 * sHw_wHs), sc, wHw);
                     } else if (__all_sync(0xFFFFFFFFu, zero)) {
                         E = E_zero;
                     } else {
-                    float2 dw[8];
+                        float2 dw[8];
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        // q = min(RNE of u on the grid 2^k {0,.5,1,1.5,2,3,4,6,...}, 6 * 2^k): the
-                        // magic constant M = 1.5 * 2^23 * spacing comes from the binade of u
-                        // clamped to [2^k, 4 * 2^k]; (u + M) - M rounds u to the spacing with
-                        // ties to even, and values past 6 * 2^k land at or above it.
-                        const float2 M = make_float2(__uint_as_float(min(max(ep[2 * p], mlo), mhi)),
-                                                     __uint_as_float(min(max(ep[2 * p + 1], mlo), mhi)));
-                        const float2 t = __fadd2_rn(u[p], M);
-                        float2 q = __ffma2_rn(M, make_float2(-1.0f, -1.0f), t);  // t - M, exact
-                        q.x = fminf(q.x, lim);
-                        q.y = fminf(q.y, lim);
-                        dw[p] = __ffma2_rn(q, ss[p], w2[p]);  // w - q_c s_c = -dw, one rounding
-                    }
-                    // E >= mu sum_a H_aa dw_a^2: skip the form when, for every lane, that bound
-                    // (rounded down) exceeds the best so far by more than the FP32 error margin,
-                    // so the candidate can neither be the argmin nor tie it
-                    float2 lb2 = make_float2(0.0f, 0.0f);
+                        for (int p = 0; p < 8; ++p) {
+                            // q = min(RNE of u on the grid 2^k {0,.5,1,1.5,2,3,4,6,...}, 6 * 2^k): the
+                            // magic constant M = 1.5 * 2^23 * spacing comes from the binade of u
+                            // clamped to [2^k, 4 * 2^k]; (u + M) - M rounds u to the spacing with
+                            // ties to even, and values past 6 * 2^k land at or above it.
+                            const float2 M = make_float2(__uint_as_float(min(max(ep[2 * p], mlo), mhi)),
+                                                         __uint_as_float(min(max(ep[2 * p + 1], mlo), mhi)));
+                            const float2 t = __fadd2_rn(u[p], M);
+                            float2 q = __ffma2_rn(M, make_float2(-1.0f, -1.0f), t);  // t - M, exact
+                            q.x = fminf(q.x, lim);
+                            q.y = fminf(q.y, lim);
+                            dw[p] = __ffma2_rn(q, ss[p], w2[p]);  // w - q_c s_c = -dw, one rounding
+                        }
+                        // E >= mu sum_a H_aa dw_a^2: skip the form when, for every lane, that bound
+                        // (rounded down) exceeds the best so far by more than the FP32 error margin,
+                        // so the candidate can neither be the argmin nor tie it
+                        float2 lb2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                    for (int p = 0; p < 8; p += 2) {
-                        const float4 d4 = lds128(&sm.dg[p]);
-                        lb2 = __ffma2_rn(__fmul2_rn(dw[p], dw[p]), make_float2(d4.x, d4.y), lb2);
-                        lb2 = __ffma2_rn(__fmul2_rn(dw[p + 1], dw[p + 1]), make_float2(d4.z, d4.w), lb2);
-                    }
-                    const float LB = (lb2.x + lb2.y) * mu_lb;
-                    if (__all_sync(0xFFFFFFFFu, LB > best_e + margin)) E = __int_as_float(0x7F800000);
-                    else E = form(dw);
+                        for (int p = 0; p < 8; p += 2) {
+                            const float4 d4 = lds128(&sm.dg[p]);
+                            lb2 = __ffma2_rn(__fmul2_rn(dw[p], dw[p]), make_float2(d4.x, d4.y), lb2);
+                            lb2 = __ffma2_rn(__fmul2_rn(dw[p + 1], dw[p + 1]), make_float2(d4.z, d4.w), lb2);
+                        }
+                        const float thr = best_e + margin;
+                        const float LB = (lb2.x + lb2.y) * mu_lb;
+                        if (__all_sync(0xFFFFFFFFu, LB > thr)) {
+                            E = __int_as_float(0x7F800000);
+                            // the same bound over this pass's tail set only: zeroed weights
+                            // (u <= 2^k / 4) going up, saturated ones (u > 5 * 2^k) going down
+                            const float tt = up ? __int_as_float((125 + k) << 23)
+                                                : __int_as_float(((129 + k) << 23) | 0x200000);
+                            float2 tl2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+                            for (int p = 0; p < 8; p += 2) {
+                                const float4 d4 = lds128(&sm.dg[p]);
+                                const float2 s0q = __fmul2_rn(dw[p], dw[p]), s1q = __fmul2_rn(dw[p + 1], dw[p + 1]);
+                                const float2 m0 = make_float2(((u[p].x > tt) != up) ? s0q.x : 0.0f,
+                                                              ((u[p].y > tt) != up) ? s0q.y : 0.0f);
+                                const float2 m1 = make_float2(((u[p + 1].x > tt) != up) ? s1q.x : 0.0f,
+                                                              ((u[p + 1].y > tt) != up) ? s1q.y : 0.0f);
+                                tl2 = __ffma2_rn(m0, make_float2(d4.x, d4.y), tl2);
+                                tl2 = __ffma2_rn(m1, make_float2(d4.z, d4.w), tl2);
+                            }
+                            stop = __all_sync(0xFFFFFFFFu, (tl2.x + tl2.y) * mu_lb > thr);
+                        } else {
+                            E = form(dw);
+                        }
                     }
                     if (E < best_e) {
                         second_e = best_e;
@@ -500,7 +527,23 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     } else {
                         second_e = fminf(second_e, E);
                     }
+                    return stop;
+                };
+                // start at the warp's mean max-scaling index (6 * 2^k >= max u)
+                int kst = 0;
+                {
+                    const float x = umax * 0.16666667f;
+                    const int e = (int)((__float_as_uint(x) >> 23) & 0xFF) - 127;
+                    kst = (x > 1.0f) ? e + ((__float_as_uint(x) & 0x7FFFFF) ? 1 : 0) : 0;
+                    kst = max(0, min(n - 1, kst));
                 }
+                const int k0 = (int)((__reduce_add_sync(0xFFFFFFFFu, (unsigned)kst) + 16u) >> 5);
+#pragma unroll 1
+                for (int k = k0; k < n; ++k)
+                    if (candidate(k, true)) break;
+#pragma unroll 1
+                for (int k = k0 - 1; k >= 0; --k)
+                    if (candidate(k, false)) break;
             }
             // Exact FP32 ties (second == best) are flagged too, so the FP64 re-sweep applies
             // the lowest-code rule.
