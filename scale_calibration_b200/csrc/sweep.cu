@@ -85,7 +85,7 @@ __device__ __forceinline__ float div_by_recip(float a, float b, float y) {
 
 // FP64 error of candidate code c for block w (definition order of the method:
 // s = fp32(v(c) g), q = E2M1(fp32(w/s)), dw = q s - w exact, E = dw^T H dw).
-__device__ double candidate_error_f64(const float (&w)[16], float g, int c, const float* Hf) {
+__device__ __noinline__ double candidate_error_f64(const float (&w)[16], float g, int c, const float* Hf) {
     const float s = __fmul_rn(e4m3_value(c), g);
     double dw[16];
 #pragma unroll
@@ -538,12 +538,18 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     kst = max(0, min(n - 1, kst));
                 }
                 const int k0 = (int)((__reduce_add_sync(0xFFFFFFFFu, (unsigned)kst) + 16u) >> 5);
+                // one loop for both directions keeps a single copy of the candidate code
+                bool up = true;
+                int k = k0;
 #pragma unroll 1
-                for (int k = k0; k < n; ++k)
-                    if (candidate(k, true)) break;
-#pragma unroll 1
-                for (int k = k0 - 1; k >= 0; --k)
-                    if (candidate(k, false)) break;
+                while (true) {
+                    if (up && k >= n) { up = false; k = k0 - 1; }
+                    if (!up && k < 0) break;
+                    const bool stop = candidate(k, up);
+                    if (stop && up) { up = false; k = k0 - 1; continue; }
+                    if (stop) break;
+                    k += up ? 1 : -1;
+                }
             }
             // Exact FP32 ties (second == best) are flagged too, so the FP64 re-sweep applies
             // the lowest-code rule.
