@@ -83,6 +83,13 @@ __device__ __forceinline__ float div_by_recip(float a, float b, float y) {
     return __fmaf_rn(r, y, q);
 }
 
+// IEEE quotients |w_i| / s0 for blocks holding a tiny non-zero weight (rare;
+// kept out of line so the hot loop stays small).
+__device__ __noinline__ void quotients_ieee(const float (&w)[16], float s0, float2 (&u)[8]) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) u[p] = make_float2(__fdiv_rn(fabsf(w[2 * p]), s0), __fdiv_rn(fabsf(w[2 * p + 1]), s0));
+}
+
 // FP64 error of candidate code c for block w (definition order of the method:
 // s = fp32(v(c) g), q = E2M1(fp32(w/s)), dw = q s - w exact, E = dw^T H dw).
 __device__ __noinline__ double candidate_error_f64(const float (&w)[16], float g, int c, const float* Hf) {
@@ -432,13 +439,18 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 float2 u[8], ss[8];
                 unsigned ep[16];
                 float umin = __int_as_float(0x7F800000), umax = 0.0f;  // over the non-zero weights
-                const float rs0 = __frcp_rn(s0);
+                if (tiny_w) {
+                    quotients_ieee(w, s0, u);
+                } else {
+                    const float rs0 = __frcp_rn(s0);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p)
+                        u[p] = make_float2(div_by_recip(fabsf(w[2 * p]), s0, rs0),
+                                           div_by_recip(fabsf(w[2 * p + 1]), s0, rs0));
+                }
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {
-                    const float u0 = tiny_w ? __fdiv_rn(fabsf(w[2 * p]), s0) : div_by_recip(fabsf(w[2 * p]), s0, rs0);
-                    const float u1 = tiny_w ? __fdiv_rn(fabsf(w[2 * p + 1]), s0)
-                                            : div_by_recip(fabsf(w[2 * p + 1]), s0, rs0);
-                    u[p] = make_float2(u0, u1);
+                    const float u0 = u[p].x, u1 = u[p].y;
                     // -sign(w) s0: the form is even in dw, so w - q s (= -dw) is used
                     ss[p] = make_float2(copysignf(s0, -w[2 * p]), copysignf(s0, -w[2 * p + 1]));
                     ep[2 * p] = (__float_as_uint(u0) & 0x7F800000u) + 0x0B400000u;
