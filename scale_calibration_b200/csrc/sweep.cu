@@ -398,6 +398,14 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             // |E32 - E| <= 30 u T <= 30 u Tw per candidate (u = 2^-24); 48 u leaves slack
             // for the rounding of Tw itself.
             const float margin = 2.0f * (48.0f * 5.9604645e-8f) * Tw;
+            // With mu > 0, H is positive semidefinite, so |H_ab| <= sqrt(H_aa H_bb) and
+            // T <= (sum_a sqrt(H_aa) |dw_a|)^2 <= 16 sum_a H_aa dw_a^2 <= 16 E / mu: the FP32
+            // error becomes relative, |E32 - E| <= rho E with rho = 16 * 48 u / mu, far tighter
+            // than the Tw bound for the candidates near the optimum. Thresholds then follow
+            // from E in [E32 / (1 + rho), E32 / (1 - rho)]; closed forms are within 2u.
+            const bool rel = sm.mu > 0.0f;
+            const float rho = rel ? fminf(768.0f * 5.9604645e-8f / sm.mu * 1.001f, 0.25f) : 0.0f;
+            const float up_fac = 1.0f / (1.0f - rho) * (1.0f + 4.0f * 5.9604645e-8f);  // E* <= E32 * up_fac
             // mu rounded down, less 32 u for the rounding of dw and of the bound's sum
             const float mu_lb = sm.mu * (1.0f - 32.0f * 5.9604645e-8f);
             // Closed forms in FP64 with sigma = sign(w) (0 where w = 0): a saturated
@@ -507,7 +515,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                             lb2 = __ffma2_rn(__fmul2_rn(dw[p], dw[p]), make_float2(d4.x, d4.y), lb2);
                             lb2 = __ffma2_rn(__fmul2_rn(dw[p + 1], dw[p + 1]), make_float2(d4.z, d4.w), lb2);
                         }
-                        const float thr = best_e + margin;
+                        // a candidate is out once its exact error provably exceeds the incumbent's
+                        // (only when mu > 0: otherwise E may be negative and nothing is pruned)
+                        const float thr = rel ? best_e * up_fac : __int_as_float(0x7F800000);
                         const float LB = (lb2.x + lb2.y) * mu_lb;
                         if (__all_sync(0xFFFFFFFFu, LB > thr)) {
                             E = __int_as_float(0x7F800000);
@@ -565,7 +575,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             }
             // Exact FP32 ties (second == best) are flagged too, so the FP64 re-sweep applies
             // the lowest-code rule.
-            if (!(second_e - best_e > margin)) flag = true;  // also catches NaN / inf
+            const bool clear = rel ? (second_e * (1.0f - 4.0f * 5.9604645e-8f) > best_e * up_fac * (1.0f + rho))
+                                   : (second_e - best_e > margin);
+            if (!clear) flag = true;  // also catches NaN / inf
         }
 
         // FP64 re-sweep of flagged blocks, one block at a time across the warp.

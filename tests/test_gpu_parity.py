@@ -216,3 +216,26 @@ def test_tiny_weights_inside_normal_blocks(cuda_ok):
     idx = rng.choice(W.size, size=W.size // 8, replace=False)
     W.reshape(-1)[idx] *= np.float32(10.0) ** rng.integers(-36, -2, size=idx.size).astype(np.float32)
     _full_parity(layer)
+
+
+def test_indefinite_hessian_gets_exact_argmin(cuda_ok):
+    # a symmetric but indefinite H (errors can be negative): no pruning may apply,
+    # the sweep must still return the oracle's argmin
+    import scale_calibration_b200 as lh
+    layer = synth.make_layer(96, 64, 10, seed=15, w_dtype="f32")
+    W, _, _ = gu.to_device(layer)
+    rng = np.random.default_rng(15)
+    Hn = np.zeros((1, 4, 16, 16), np.float32)
+    for j in range(4):
+        A = rng.standard_normal((16, 16)).astype(np.float32)
+        Hn[0, j] = (A + A.T) * np.float32(0.5)
+    H = torch.from_numpy(Hn).cuda()
+    amax = torch.empty(1, device="cuda")
+    lh.lh_absmax(W, W, 1, 96, 64, 64, amax)
+    codes = torch.empty(1, 96, 4, dtype=torch.uint8, device="cuda")
+    bam = torch.empty(1, 96, 4, device="cuda")
+    lh.lh_sweep_scales(W, W, 1, 96, 64, 64, amax, H, bam, codes)
+    torch.cuda.synchronize()
+    ex, tol, fail, worst = gu.check_codes(layer.W_f32(), amax.cpu().numpy(), Hn.astype(np.float64),
+                                          codes.cpu().numpy(), bam.cpu().numpy())
+    assert fail == 0, (ex, tol, fail, worst)
