@@ -383,36 +383,40 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         if (g == 0.0f) flag = false;  // every s_c is 0: q = 0, all errors equal, code 1
 
         if (fast) {
-            // Tw = sum_{a<=b} |U_ab| |w_a| |w_b| bounds sum |U_ab| |dw_a| |dw_b| for every candidate.
-            float Tw = 0.0f;
-#pragma unroll
-            for (int a = 0; a < 16; ++a) {
-                float t = sm.Ua[tri(a, a)] * fabsf(w[a]);
-#pragma unroll
-                for (int b = a + 1; b < 16; ++b) t = fmaf(sm.Ua[tri(a, b)], fabsf(w[b]), t);
-                Tw = fmaf(fabsf(w[a]), t, Tw);
-            }
-            float2 w2[8];
-#pragma unroll
-            for (int p = 0; p < 8; ++p) w2[p] = make_float2(w[2 * p], w[2 * p + 1]);
-            // |E32 - E| <= 30 u T <= 30 u Tw per candidate (u = 2^-24); 48 u leaves slack
-            // for the rounding of Tw itself.
-            const float margin = 2.0f * (48.0f * 5.9604645e-8f) * Tw;
             // With mu > 0, H is positive semidefinite, so |H_ab| <= sqrt(H_aa H_bb) and
             // T <= (sum_a sqrt(H_aa) |dw_a|)^2 <= 16 sum_a H_aa dw_a^2 <= 16 E / mu: the FP32
             // error becomes relative, |E32 - E| <= rho E with rho = 16 * 48 u / mu, far tighter
-            // than the Tw bound for the candidates near the optimum. Thresholds then follow
-            // from E in [E32 / (1 + rho), E32 / (1 - rho)]; closed forms are within 2u.
+            // than the Tw bound below for the candidates near the optimum. Thresholds then
+            // follow from E in [E32 / (1 + rho), E32 / (1 - rho)]; closed forms are within 2u.
             const bool rel = sm.mu > 0.0f;
             const float rho = rel ? fminf(768.0f * 5.9604645e-8f / sm.mu * 1.001f, 0.25f) : 0.0f;
             const float up_fac = 1.0f / (1.0f - rho) * (1.0f + 4.0f * 5.9604645e-8f);  // E* <= E32 * up_fac
             // mu rounded down, less 32 u for the rounding of dw and of the bound's sum
             const float mu_lb = sm.mu * (1.0f - 32.0f * 5.9604645e-8f);
+            // Without mu: Tw = sum_{a<=b} |U_ab| |w_a| |w_b| bounds sum |U_ab| |dw_a| |dw_b| for
+            // every candidate, and |E32 - E| <= 30 u T <= 30 u Tw (48 u leaves slack for the
+            // rounding of Tw itself).
+            float margin = 0.0f;
+            if (!rel) {
+                float Tw = 0.0f;
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    float t = sm.Ua[tri(a, a)] * fabsf(w[a]);
+#pragma unroll
+                    for (int b = a + 1; b < 16; ++b) t = fmaf(sm.Ua[tri(a, b)], fabsf(w[b]), t);
+                    Tw = fmaf(fabsf(w[a]), t, Tw);
+                }
+                margin = 2.0f * (48.0f * 5.9604645e-8f) * Tw;
+            }
+            float2 w2[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) w2[p] = make_float2(w[2 * p], w[2 * p + 1]);
             // Closed forms in FP64 with sigma = sign(w) (0 where w = 0): a saturated
             // candidate has dw = 6 s_c sigma - w, so E = 36 s^2 sHs - 6 s (sHw + wHs) + wHw;
-            // an all-zero candidate has dw = -w, so E = wHw.
+            // an all-zero candidate has dw = -w, so E = wHw. Formed on first use.
             double sHs = 0.0, sHw_wHs = 0.0, wHw = 0.0;
-            {
+            bool have_cf = false;
+            auto closed_form_coeffs = [&]() {
                 double wd[16], sd[16];
 #pragma unroll
                 for (int a = 0; a < 16; ++a) {
@@ -432,8 +436,8 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     sHs = fma(sd[a], ts, sHs);
                     sHw_wHs = fma(sd[a], tw, fma(wd[a], ts, sHw_wHs));
                 }
-            }
-            const float E_zero = (float)wHw;
+                have_cf = true;
+            };
             // the reciprocal-based quotient needs every non-zero |w| >= 2^-100
             const bool tiny_w = __uint_as_float((uint32_t)(sm.order[rr * kThreads + tid] >> 32)) < 7.888609e-31f;
 
@@ -484,11 +488,11 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     const bool zero = umax <= __int_as_float((125 + k) << 23);              // 2^k / 4
                     float E;
                     bool stop = false;
-                    if (__all_sync(0xFFFFFFFFu, sat)) {
+                    const bool all_sat = __all_sync(0xFFFFFFFFu, sat);
+                    if (all_sat || __all_sync(0xFFFFFFFFu, zero)) {
+                        if (!have_cf) closed_form_coeffs();
                         const double sc = (double)s0 * (double)__int_as_float((127 + k) << 23);  // s_c, exact
-                        E = (float)fma(fma(36.0 * sHs, sc, -6.0 * sHw_wHs), sc, wHw);
-                    } else if (__all_sync(0xFFFFFFFFu, zero)) {
-                        E = E_zero;
+                        E = all_sat ? (float)fma(fma(36.0 * sHs, sc, -6.0 * sHw_wHs), sc, wHw) : (float)wHw;
                     } else {
                         float2 dw[8];
 #pragma unroll
