@@ -230,7 +230,7 @@ __device__ __forceinline__ float quad_form_smem(const float2 (&dw)[8], const Swe
 }
 
 template <typename T, bool kURegs>
-__global__ void __launch_bounds__(kThreads, kURegs ? 2 : 3)
+__global__ void __launch_bounds__(kThreads, kURegs ? 2 : 4)
 sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int64_t mat_stride,
              const float* __restrict__ gamax, const float* __restrict__ H, float* __restrict__ best_amax,
              uint8_t* __restrict__ best_code) {
@@ -512,13 +512,14 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         // E >= mu sum_a H_aa dw_a^2: skip the form when, for every lane, that bound
                         // (rounded down) exceeds the best so far by more than the FP32 error margin,
                         // so the candidate can neither be the argmin nor tie it
-                        float2 lb2 = make_float2(0.0f, 0.0f);
+                        float2 lb2 = make_float2(0.0f, 0.0f), lb2b = make_float2(0.0f, 0.0f);  // two chains
 #pragma unroll
                         for (int p = 0; p < 8; p += 2) {
                             const float4 d4 = lds128(&sm.dg[p]);
                             lb2 = __ffma2_rn(__fmul2_rn(dw[p], dw[p]), make_float2(d4.x, d4.y), lb2);
-                            lb2 = __ffma2_rn(__fmul2_rn(dw[p + 1], dw[p + 1]), make_float2(d4.z, d4.w), lb2);
+                            lb2b = __ffma2_rn(__fmul2_rn(dw[p + 1], dw[p + 1]), make_float2(d4.z, d4.w), lb2b);
                         }
+                        lb2 = __fadd2_rn(lb2, lb2b);
                         // a candidate is out once its exact error provably exceeds the incumbent's
                         // (only when mu > 0: otherwise E may be negative and nothing is pruned)
                         const float thr = rel ? best_e * up_fac : __int_as_float(0x7F800000);
