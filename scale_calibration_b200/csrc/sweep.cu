@@ -83,29 +83,31 @@ __device__ __forceinline__ float div_by_recip(float a, float b, float y) {
     return __fmaf_rn(r, y, q);
 }
 
-// IEEE quotients |w_i| / s0 for blocks holding a tiny non-zero weight (rare;
+// IEEE quotients w_i / s0 for blocks holding a tiny non-zero weight (rare;
 // kept out of line so the hot loop stays small).
 __device__ __noinline__ void quotients_ieee(const float (&w)[16], float s0, float2 (&u)[8]) {
 #pragma unroll
-    for (int p = 0; p < 8; ++p) u[p] = make_float2(__fdiv_rn(fabsf(w[2 * p]), s0), __fdiv_rn(fabsf(w[2 * p + 1]), s0));
+    for (int p = 0; p < 8; ++p) u[p] = make_float2(__fdiv_rn(w[2 * p], s0), __fdiv_rn(w[2 * p + 1], s0));
 }
 
 // FP64 error of candidate code c for block w (definition order of the method:
-// s = fp32(v(c) g), q = E2M1(fp32(w/s)), dw = q s - w exact, E = dw^T H dw).
-__device__ __noinline__ double candidate_error_f64(const float (&w)[16], float g, int c, const float* Hf) {
+// s = fp32(v(c) g), q = E2M1(fp32(w/s)), dw = q s - w exact, E = dw^T H dw),
+// the form taken over the packed upper triangle Us (H_aa, H_ab + H_ba in FP64).
+__device__ __noinline__ double candidate_error_f64(const float (&w)[16], float g, int c, const double* Us) {
     const float s = __fmul_rn(e4m3_value(c), g);
+    const double sd = (double)s;
     double dw[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const float q = (s != 0.0f) ? e2m1_rne(__fdiv_rn(w[i], s)) : 0.0f;
-        dw[i] = (double)q * (double)s - (double)w[i];
+        dw[i] = fma((double)q, sd, -(double)w[i]);  // q s - w: q s has at most 27 significant bits
     }
     double E = 0.0;
 #pragma unroll 1
     for (int a = 0; a < 16; ++a) {
         double t = 0.0;
 #pragma unroll
-        for (int b = 0; b < 16; ++b) t = fma((double)Hf[a * 16 + b], dw[b], t);
+        for (int b = 15; b >= a; --b) t = fma(Us[tri(a, b)], dw[b], t);
         E = fma(dw[a], t, E);
     }
     return E;
@@ -378,7 +380,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         }
 
         float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
-        int best_c = 1;
+        int best_fk = -1;  // 32 f + k of the best candidate (class f, step k); the code is formed at the end
         bool flag = !fast;
         if (g == 0.0f) flag = false;  // every s_c is 0: q = 0, all errors equal, code 1
 
@@ -411,33 +413,19 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             float2 w2[8];
 #pragma unroll
             for (int p = 0; p < 8; ++p) w2[p] = make_float2(w[2 * p], w[2 * p + 1]);
-            // Closed forms in FP64 with sigma = sign(w) (0 where w = 0): a saturated
-            // candidate has dw = 6 s_c sigma - w, so E = 36 s^2 sHs - 6 s (sHw + wHs) + wHw;
-            // an all-zero candidate has dw = -w, so E = wHw. Formed on first use.
-            double sHs = 0.0, sHw_wHs = 0.0, wHw = 0.0;
-            bool have_cf = false;
-            auto closed_form_coeffs = [&]() {
-                double wd[16], sd[16];
+            // the upward bound loses at most 2^-22 H_aa w_a^2 per weight to the rounding of u;
+            // 2^-20 mu sum_a H_aa w_a^2 covers it with room for the rounding of the sum
+            float tail_corr;
+            {
+                float2 sw = make_float2(0.0f, 0.0f);
 #pragma unroll
-                for (int a = 0; a < 16; ++a) {
-                    wd[a] = (double)w[a];
-                    sd[a] = (w[a] > 0.0f) ? 1.0 : (w[a] < 0.0f ? -1.0 : 0.0);
+                for (int p = 0; p < 8; p += 2) {
+                    const float4 d4 = lds128(&sm.dg[p]);
+                    sw = __ffma2_rn(__fmul2_rn(w2[p], w2[p]), make_float2(d4.x, d4.y), sw);
+                    sw = __ffma2_rn(__fmul2_rn(w2[p + 1], w2[p + 1]), make_float2(d4.z, d4.w), sw);
                 }
-#pragma unroll
-                for (int a = 0; a < 16; ++a) {
-                    double tw = 0.0, ts = 0.0;  // sum_{b >= a} Us_ab w_b, Us_ab sigma_b
-#pragma unroll
-                    for (int b = a; b < 16; ++b) {
-                        const double h = sm.Us[tri(a, b)];
-                        tw = fma(h, wd[b], tw);
-                        ts = fma(h, sd[b], ts);
-                    }
-                    wHw = fma(wd[a], tw, wHw);
-                    sHs = fma(sd[a], ts, sHs);
-                    sHw_wHs = fma(sd[a], tw, fma(wd[a], ts, sHw_wHs));
-                }
-                have_cf = true;
-            };
+                tail_corr = (sw.x + sw.y) * (sm.mu * 9.5367432e-7f);  // 2^-20 mu
+            }
             // the reciprocal-based quotient needs every non-zero |w| >= 2^-100
             const bool tiny_w = __uint_as_float((uint32_t)(sm.order[rr * kThreads + tid] >> 32)) < 7.888609e-31f;
 
@@ -448,67 +436,92 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 const int n = (f == 7 ? 7 : 8) - x0 + 1;  // codes in the class
                 const float v0 = (float)(8 + f) * __int_as_float((x0 - 3 + 127) << 23);  // (1 + f/8) 2^x0
                 const float s0 = __fmul_rn(v0, g);
-                float2 u[8], ss[8];
+                // signed quotients u = w / s0; candidate k of the class has the scale 2^k s0
+                float2 u[8];
                 unsigned ep[16];
-                float umin = __int_as_float(0x7F800000), umax = 0.0f;  // over the non-zero weights
+                float umax = 0.0f;  // max |u|
                 if (tiny_w) {
                     quotients_ieee(w, s0, u);
                 } else {
                     const float rs0 = __frcp_rn(s0);
 #pragma unroll
                     for (int p = 0; p < 8; ++p)
-                        u[p] = make_float2(div_by_recip(fabsf(w[2 * p]), s0, rs0),
-                                           div_by_recip(fabsf(w[2 * p + 1]), s0, rs0));
+                        u[p] = make_float2(div_by_recip(w[2 * p], s0, rs0), div_by_recip(w[2 * p + 1], s0, rs0));
                 }
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {
-                    const float u0 = u[p].x, u1 = u[p].y;
-                    // -sign(w) s0: the form is even in dw, so w - q s (= -dw) is used
-                    ss[p] = make_float2(copysignf(s0, -w[2 * p]), copysignf(s0, -w[2 * p + 1]));
-                    ep[2 * p] = (__float_as_uint(u0) & 0x7F800000u) + 0x0B400000u;
-                    ep[2 * p + 1] = (__float_as_uint(u1) & 0x7F800000u) + 0x0B400000u;
-                    umin = (w[2 * p] != 0.0f) ? fminf(umin, u0) : umin;
-                    umin = (w[2 * p + 1] != 0.0f) ? fminf(umin, u1) : umin;
-                    umax = fmaxf(umax, fmaxf(u0, u1));
+                    ep[2 * p] = (__float_as_uint(u[p].x) & 0x7F800000u) + 0x0B400000u;
+                    ep[2 * p + 1] = (__float_as_uint(u[p].y) & 0x7F800000u) + 0x0B400000u;
+                    umax = fmaxf(umax, fmaxf(fabsf(u[p].x), fabsf(u[p].y)));
                 }
-                // One candidate; returns true when every lane proves that the rest of this
-                // pass is prunable. Pass 0 walks k upwards: the weights quantised to zero
-                // (dw_i = w_i exactly) only grow in number, so mu * sum_{q_i = 0} H_ii w_i^2
-                // bounds every later candidate. Pass 1 walks k downwards: saturated weights
-                // stay saturated and their |dw_i| = | |w_i| - 6 s_c | only grows as s_c
-                // halves, so mu * sum_{saturated} H_ii dw_i^2 bounds every later candidate.
+                const float2 ns0 = make_float2(-s0, -s0);
+                // One candidate; returns true (upward walk only) when every lane proves that no
+                // later candidate of the upward walk can beat the incumbent.
                 auto candidate = [&](int k, bool up) -> bool {
-                    const int code = class_code(f, x0 + k);
                     const float lim = __int_as_float(((129 + k) << 23) | 0x400000);  // 6 * 2^k
                     const unsigned mlo = ((unsigned)(127 + k) << 23) + 0x0B400000u;
-                    const unsigned mhi = ((unsigned)(129 + k) << 23) + 0x0B400000u;
-                    // every non-zero weight saturates (q = +-6) iff min u > 5 * 2^k; every q is 0
-                    // iff max u <= 2^k / 4 (ties 5 -> 4 and 1/4 -> 0 round to even)
-                    const bool sat = umin > __int_as_float(((129 + k) << 23) | 0x200000);  // 5 * 2^k
-                    const bool zero = umax <= __int_as_float((125 + k) << 23);              // 2^k / 4
                     float E;
-                    bool stop = false;
-                    const bool all_sat = __all_sync(0xFFFFFFFFu, sat);
-                    if (all_sat || __all_sync(0xFFFFFFFFu, zero)) {
-                        if (!have_cf) closed_form_coeffs();
-                        const double sc = (double)s0 * (double)__int_as_float((127 + k) << 23);  // s_c, exact
-                        E = all_sat ? (float)fma(fma(36.0 * sHs, sc, -6.0 * sHw_wHs), sc, wHw) : (float)wHw;
-                    } else {
-                        float2 dw[8];
+                    bool stop = false, done = false;
+                    if (!rel) {
+                        // no pruning here, so whole-block shortcuts pay: every non-zero weight
+                        // saturates (q = +-6) iff min |u| > 5 * 2^k; every q is 0 iff max |u| <= 2^k / 4
+                        // (ties 5 -> 4 and 1/4 -> 0 round to even)
+                        float umin = __int_as_float(0x7F800000);
 #pragma unroll
                         for (int p = 0; p < 8; ++p) {
-                            // q = min(RNE of u on the grid 2^k {0,.5,1,1.5,2,3,4,6,...}, 6 * 2^k): the
-                            // magic constant M = 1.5 * 2^23 * spacing comes from the binade of u
-                            // clamped to [2^k, 4 * 2^k]; (u + M) - M rounds u to the spacing with
-                            // ties to even, and values past 6 * 2^k land at or above it.
-                            const float2 M = make_float2(__uint_as_float(min(max(ep[2 * p], mlo), mhi)),
-                                                         __uint_as_float(min(max(ep[2 * p + 1], mlo), mhi)));
-                            const float2 t = __fadd2_rn(u[p], M);
-                            float2 q = __ffma2_rn(M, make_float2(-1.0f, -1.0f), t);  // t - M, exact
-                            q.x = fminf(q.x, lim);
-                            q.y = fminf(q.y, lim);
-                            dw[p] = __ffma2_rn(q, ss[p], w2[p]);  // w - q_c s_c = -dw, one rounding
+                            umin = (w2[p].x != 0.0f) ? fminf(umin, fabsf(u[p].x)) : umin;
+                            umin = (w2[p].y != 0.0f) ? fminf(umin, fabsf(u[p].y)) : umin;
                         }
+                        const bool sat = umin > __int_as_float(((129 + k) << 23) | 0x200000);  // 5 * 2^k
+                        const bool zero = umax <= __int_as_float((125 + k) << 23);              // 2^k / 4
+                        const bool all_sat = __all_sync(0xFFFFFFFFu, sat);
+                        if (all_sat || __all_sync(0xFFFFFFFFu, zero)) {
+                            // closed forms in FP64 with sigma = sign(w) (0 where w = 0): a saturated
+                            // candidate has dw = 6 s_c sigma - w, so E = 36 s^2 sHs - 6 s (sHw + wHs) + wHw;
+                            // an all-zero candidate has dw = -w, so E = wHw
+                            double sHs = 0.0, sHw_wHs = 0.0, wHw = 0.0;
+#pragma unroll 1
+                            for (int a = 0; a < 16; ++a) {
+                                const double wa = (double)w[a];
+                                const double sa = (w[a] > 0.0f) ? 1.0 : (w[a] < 0.0f ? -1.0 : 0.0);
+                                double tw = 0.0, ts = 0.0;  // sum_{b >= a} Us_ab w_b, Us_ab sigma_b
+                                for (int b = a; b < 16; ++b) {
+                                    const double h = sm.Us[tri(a, b)];
+                                    tw = fma(h, (double)w[b], tw);
+                                    ts = fma(h, (w[b] > 0.0f) ? 1.0 : (w[b] < 0.0f ? -1.0 : 0.0), ts);
+                                }
+                                wHw = fma(wa, tw, wHw);
+                                sHs = fma(sa, ts, sHs);
+                                sHw_wHs = fma(sa, tw, fma(wa, ts, sHw_wHs));
+                            }
+                            const double sc = (double)s0 * (double)__int_as_float((127 + k) << 23);  // s_c, exact
+                            E = all_sat ? (float)fma(fma(36.0 * sHs, sc, -6.0 * sHw_wHs), sc, wHw) : (float)wHw;
+                            done = true;
+                        }
+                    }
+                    if (!done) {
+                        // q = RNE of u on the grid 2^k {0,.5,1,1.5,2,3,4,6,8,12,...}: the magic
+                        // constant M = 1.5 * 2^23 * spacing comes from the binade of |u|, raised to
+                        // that of 2^k; (u + M) - M rounds u to the spacing with ties to even (the
+                        // grid is symmetric, so the sign rides along). Values past 6 * 2^k land at
+                        // or beyond it and are clamped, in warps that hold any.
+                        float2 q[8];
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+                            const float2 M = make_float2(__uint_as_float(max(ep[2 * p], mlo)),
+                                                         __uint_as_float(max(ep[2 * p + 1], mlo)));
+                            q[p] = __ffma2_rn(M, make_float2(-1.0f, -1.0f), __fadd2_rn(u[p], M));  // exact
+                        }
+                        if (__any_sync(0xFFFFFFFFu, umax > lim)) {
+#pragma unroll
+                            for (int p = 0; p < 8; ++p) {
+                                q[p].x = fminf(fmaxf(q[p].x, -lim), lim);
+                                q[p].y = fminf(fmaxf(q[p].y, -lim), lim);
+                            }
+                        }
+                        float2 dw[8];
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) dw[p] = __ffma2_rn(q[p], ns0, w2[p]);  // w - q_c s_c = -dw, one rounding
                         // E >= mu sum_a H_aa dw_a^2: skip the form when, for every lane, that bound
                         // (rounded down) exceeds the best so far by more than the FP32 error margin,
                         // so the candidate can neither be the argmin nor tie it
@@ -523,26 +536,34 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         // a candidate is out once its exact error provably exceeds the incumbent's
                         // (only when mu > 0: otherwise E may be negative and nothing is pruned)
                         const float thr = rel ? best_e * up_fac : __int_as_float(0x7F800000);
-                        const float LB = (lb2.x + lb2.y) * mu_lb;
-                        if (__all_sync(0xFFFFFFFFu, LB > thr)) {
+                        const float lbraw = lb2.x + lb2.y;
+                        if (__all_sync(0xFFFFFFFFu, lbraw * mu_lb > thr)) {
                             E = __int_as_float(0x7F800000);
-                            // the same bound over this pass's tail set only: zeroed weights
-                            // (u <= 2^k / 4) going up, saturated ones (u > 5 * 2^k) going down
-                            const float tt = up ? __int_as_float((125 + k) << 23)
-                                                : __int_as_float(((129 + k) << 23) | 0x200000);
-                            float2 tl2 = make_float2(0.0f, 0.0f);
+                            if (up) {
+                                // Every larger scale of the class, 2^k' s0 with k' > k, has its grid
+                                // points in {0, .5, 1, 1.5, 2, 3, 4, 6, 8, 12, ...} 2^k, so a weight
+                                // with |w| / s0 <= 7 * 2^k stays at least its distance to the grid at
+                                // k, |dw| here, away from it (less 2^-23 |w| for the rounding of u).
+                                // Weights at or past 7 * 2^k count zero.
+                                const float c7 = __int_as_float(((129 + k) << 23) | 0x5FFFFD);  // 7 * 2^k (1 - 2^-22)
+                                float tail = lbraw;
+                                if (!__all_sync(0xFFFFFFFFu, umax < c7)) {
+                                    float2 tl2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                            for (int p = 0; p < 8; p += 2) {
-                                const float4 d4 = lds128(&sm.dg[p]);
-                                const float2 s0q = __fmul2_rn(dw[p], dw[p]), s1q = __fmul2_rn(dw[p + 1], dw[p + 1]);
-                                const float2 m0 = make_float2(((u[p].x > tt) != up) ? s0q.x : 0.0f,
-                                                              ((u[p].y > tt) != up) ? s0q.y : 0.0f);
-                                const float2 m1 = make_float2(((u[p + 1].x > tt) != up) ? s1q.x : 0.0f,
-                                                              ((u[p + 1].y > tt) != up) ? s1q.y : 0.0f);
-                                tl2 = __ffma2_rn(m0, make_float2(d4.x, d4.y), tl2);
-                                tl2 = __ffma2_rn(m1, make_float2(d4.z, d4.w), tl2);
+                                    for (int p = 0; p < 8; p += 2) {
+                                        const float4 d4 = lds128(&sm.dg[p]);
+                                        const float2 s0q = __fmul2_rn(dw[p], dw[p]), s1q = __fmul2_rn(dw[p + 1], dw[p + 1]);
+                                        const float2 m0 = make_float2(fabsf(u[p].x) < c7 ? s0q.x : 0.0f,
+                                                                      fabsf(u[p].y) < c7 ? s0q.y : 0.0f);
+                                        const float2 m1 = make_float2(fabsf(u[p + 1].x) < c7 ? s1q.x : 0.0f,
+                                                                      fabsf(u[p + 1].y) < c7 ? s1q.y : 0.0f);
+                                        tl2 = __ffma2_rn(m0, make_float2(d4.x, d4.y), tl2);
+                                        tl2 = __ffma2_rn(m1, make_float2(d4.z, d4.w), tl2);
+                                    }
+                                    tail = tl2.x + tl2.y;
+                                }
+                                stop = __all_sync(0xFFFFFFFFu, __fmaf_rn(tail, mu_lb, -tail_corr) > thr);
                             }
-                            stop = __all_sync(0xFFFFFFFFu, (tl2.x + tl2.y) * mu_lb > thr);
                         } else {
                             E = form(dw);
                         }
@@ -550,13 +571,32 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     if (E < best_e) {
                         second_e = best_e;
                         best_e = E;
-                        best_c = code;
+                        best_fk = 32 * f + k;
                     } else {
                         second_e = fminf(second_e, E);
                     }
                     return stop;
                 };
-                // start at the warp's mean max-scaling index (6 * 2^k >= max u)
+                // Every scale 2^k' s0 with k' < k1 quantises to at most 6 * 2^k' s0 <= 3 * 2^k1 s0, so a
+                // weight with |w| > 3 * 2^k1 s0 keeps an error of at least |w| - 3 * 2^k1 s0 there: true
+                // when, for every lane, that bound already exceeds the incumbent's error.
+                auto below_excluded = [&](int k1) -> bool {
+                    if (!rel) return false;
+                    const float thr = best_e * up_fac;
+                    const float c3 = __int_as_float(((128 + k1) << 23) | 0x400000);   // 3 * 2^k1
+                    const float c3m = __int_as_float(((128 + k1) << 23) | 0x400002);  // |u| above it: |w| / s0 above 3 * 2^k1
+                    float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const float2 dg = sm.dg[p];
+                        const float d0 = fabsf(u[p].x) > c3m ? __fmaf_rn(-c3, s0, fabsf(w2[p].x)) : 0.0f;  // one rounding
+                        const float d1 = fabsf(u[p].y) > c3m ? __fmaf_rn(-c3, s0, fabsf(w2[p].y)) : 0.0f;
+                        acc0 = __fmaf_rn(d0 * d0, dg.x, acc0);
+                        acc1 = __fmaf_rn(d1 * d1, dg.y, acc1);
+                    }
+                    return __all_sync(0xFFFFFFFFu, (acc0 + acc1) * mu_lb > thr);
+                };
+                // start at the warp's mean max-scaling index (6 * 2^k >= max |u|)
                 int kst = 0;
                 {
                     const float x = umax * 0.16666667f;
@@ -565,16 +605,16 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     kst = max(0, min(n - 1, kst));
                 }
                 const int k0 = (int)((__reduce_add_sync(0xFFFFFFFFu, (unsigned)kst) + 16u) >> 5);
-                // one loop for both directions keeps a single copy of the candidate code
+                // one loop for both directions keeps a single copy of the candidate code: up
+                // from k0 until a candidate ends the upward walk, then down from k0 - 1 while
+                // the candidates below are not excluded as a whole
                 bool up = true;
                 int k = k0;
 #pragma unroll 1
                 while (true) {
                     if (up && k >= n) { up = false; k = k0 - 1; }
-                    if (!up && k < 0) break;
-                    const bool stop = candidate(k, up);
-                    if (stop && up) { up = false; k = k0 - 1; continue; }
-                    if (stop) break;
+                    if (!up && (k < 0 || below_excluded(k + 1))) break;
+                    if (candidate(k, up)) { up = false; k = k0 - 1; continue; }
                     k += up ? 1 : -1;
                 }
             }
@@ -583,6 +623,12 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             const bool clear = rel ? (second_e * (1.0f - 4.0f * 5.9604645e-8f) > best_e * up_fac * (1.0f + rho))
                                    : (second_e - best_e > margin);
             if (!clear) flag = true;  // also catches NaN / inf
+        }
+        int best_c = 1;
+        if (best_fk >= 0) {
+            const int f = best_fk >> 5;
+            const int tz = (f == 0) ? 3 : (f == 4) ? 2 : (f == 2 || f == 6) ? 1 : 0;
+            best_c = class_code(f, -6 - tz + (best_fk & 31));
         }
 
         // FP64 re-sweep of flagged blocks, one block at a time across the warp.
@@ -596,7 +642,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             double be = 0.0;
             int bc = 127;
             for (int c = lane + 1; c <= 126; c += 32) {
-                const double e = candidate_error_f64(wv, g, c, sm.Hf);
+                const double e = candidate_error_f64(wv, g, c, sm.Us);
                 if (bc == 127 || e < be) { be = e; bc = c; }
             }
 #pragma unroll
