@@ -133,7 +133,7 @@ constexpr int kTileRows = kThreads * kRowsPerThread;  // rows of one CTA, walked
 constexpr int kSortBuckets = 512;
 
 struct SweepShared {
-    unsigned long long key[kTileRows];    // (bits of min non-zero |w|) << 32 | local row
+    unsigned long long key[kTileRows];    // (bits of max |w|) << 32 | local row
     unsigned long long order[kTileRows];  // the same, grouped by sort bucket
     uint32_t hist[kSortBuckets];
     double Us[136];                     // H_aa, H_ab + H_ba (a < b) in FP64, packed upper triangle
@@ -142,42 +142,25 @@ struct SweepShared {
     float Ua[136];          // |U| packed upper triangle, for the error bound
     float Hf[256];          // H as given, for the FP64 re-sweep
     float2 dg[8];           // diagonal of H, pairs (for the lower bound)
-    float Cw[4][16][17];    // Cholesky work arrays, one per warp
-    float lcolw[4][16];
-    int pd[8];              // results of the shifted positive-definiteness tests
+    int pd[16];             // results of the shifted positive-definiteness tests
     float mu;               // mu <= lambda_min(D^-1/2 H D^-1/2), D = diag(H); 0 disables pruning
 };
 
-// Is C - mu I positive definite, C = D^-1/2 H_s D^-1/2 (H_s = (H + H^T)/2,
-// rows with H_aa = 0 replaced by identity rows)? FP32 Cholesky by one warp
-// (lane i owns row i) on its own copy `Cw`; true when every pivot is positive.
-__device__ bool shifted_pd(const float* Hf, float (*Cw)[17], float* lcol, float mu, int lane) {
-    const int i = lane;
-    const bool own = i < 16;
-    if (own) {
-        const float hii = Hf[i * 17];
-        for (int b = 0; b < 16; ++b) {
-            const float hbb = Hf[b * 17];
-            float c;
-            if (hii > 0.0f && hbb > 0.0f)
-                c = (0.5f * (Hf[i * 16 + b] + Hf[b * 16 + i])) * (rsqrtf(hii) * rsqrtf(hbb));
-            else
-                c = (i == b) ? 1.0f : 0.0f;
-            Cw[i][b] = c - ((i == b) ? mu : 0.0f);
-        }
-    }
-    __syncwarp();
+// Is C - mu I positive definite? FP32 Cholesky by one half-warp, in registers:
+// lane i (of 16) owns row i of C, and the multipliers of column k reach the
+// other rows by shuffles; true when every pivot is positive.
+__device__ __forceinline__ bool shifted_pd(const float (&crow)[16], float mu, int i) {
+    float c[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) c[b] = crow[b] - ((b == i) ? mu : 0.0f);
     bool ok = true;
+#pragma unroll
     for (int k = 0; k < 16; ++k) {
-        const float d = Cw[k][k];
+        const float d = __shfl_sync(0xFFFFFFFFu, c[k], k, 16);  // pivot, from lane k of this half
         ok = ok && (d > 0.0f);
-        const float rl = d > 0.0f ? rsqrtf(d) : 1.0f;
-        const float l_ik = (own && i > k) ? Cw[i][k] * rl : 0.0f;
-        if (own) lcol[i] = l_ik;
-        __syncwarp();
-        if (own && i > k)
-            for (int b = k + 1; b <= i; ++b) Cw[i][b] -= l_ik * lcol[b];
-        __syncwarp();
+        const float l = (i > k) ? c[k] * (d > 0.0f ? rsqrtf(d) : 1.0f) : 0.0f;  // L_ik
+#pragma unroll
+        for (int b = k + 1; b < 16; ++b) c[b] = __fmaf_rn(-l, __shfl_sync(0xFFFFFFFFu, l, b, 16), c[b]);
     }
     return ok;
 }
@@ -261,49 +244,60 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             dst[b & 1] = u;
         }
     }
-    // mu for the candidate lower bound E >= mu sum_a H_aa dw_a^2: the largest of
-    // eight shifts (two rounds, one shift per warp) at which C - mu I passes an
-    // FP32 Cholesky test. A completed factorisation is backward stable
-    // (|dC| <= 17 u |L||L^T| <= 17 u entrywise, so lambda_min(C) >= mu - 16 * 17 u);
-    // 2^-14 is subtracted to cover it. mu = 0 (no pruning) when H has a zero
-    // diagonal entry with a non-zero off-diagonal entry in its row or a negative
-    // diagonal entry, or when no shift passes.
+    // mu for the candidate lower bound E >= mu sum_a H_aa dw_a^2: the largest
+    // shift at which C - mu I passes an FP32 Cholesky test, C = D^-1/2 H_s D^-1/2
+    // (H_s = (H + H^T) / 2, D = diag(H), rows with H_aa = 0 replaced by identity
+    // rows). Two rounds of eight shifts (one per half-warp): 0.04 + 0.12 s, then
+    // nine steps up from the best of those. A completed factorisation is
+    // backward stable (|dC| <= 17 u |L||L^T| <= 17 u entrywise, so lambda_min(C)
+    // >= mu - 16 * 17 u, and forming C costs a few ulps more); 2^-14 is
+    // subtracted to cover it. mu = 0 (no pruning) when H has a zero diagonal
+    // entry with a non-zero off-diagonal entry in its row or a negative diagonal
+    // entry, or when mu would fall below 2^-8.
     {
-        bool psd_rows = true;
-        if (lane < 16) {
-            const float hii = sm.Hf[lane * 17];
-            if (!(hii >= 0.0f)) psd_rows = false;
-            if (hii == 0.0f)
-                for (int b = 0; b < 16; ++b)
-                    if (sm.Hf[lane * 16 + b] != 0.0f || sm.Hf[b * 16 + lane] != 0.0f) psd_rows = false;
-        }
+        const int hl = lane >> 4, i = lane & 15;
+        const int slot = 2 * warp + hl;  // 0..7
+        const float hii = sm.Hf[i * 17];
+        bool psd_rows = hii >= 0.0f;
+        if (hii == 0.0f)
+            for (int b = 0; b < 16; ++b)
+                if (sm.Hf[i * 16 + b] != 0.0f || sm.Hf[b * 16 + i] != 0.0f) psd_rows = false;
         psd_rows = __all_sync(0xFFFFFFFFu, psd_rows);
-        const float mu1 = 0.2f * (float)(warp + 1) - 0.1f;           // 0.1 0.3 0.5 0.7
-        const bool ok1 = psd_rows && shifted_pd(sm.Hf, sm.Cw[warp], sm.lcolw[warp], mu1, lane);
-        if (lane == 0) sm.pd[warp] = ok1;
+        const float di = hii > 0.0f ? rsqrtf(hii) : 0.0f;
+        float crow[16];
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            const float hbb = sm.Hf[b * 17];
+            const float db = __shfl_sync(0xFFFFFFFFu, di, b, 16);
+            crow[b] = (hii > 0.0f && hbb > 0.0f) ? (0.5f * (sm.Hf[i * 16 + b] + sm.Hf[b * 16 + i])) * (di * db)
+                                                 : ((i == b) ? 1.0f : 0.0f);
+        }
+        const float mu1 = 0.04f + 0.12f * (float)slot;
+        const bool ok1 = psd_rows && shifted_pd(crow, mu1, i);
+        if (i == 0) sm.pd[slot] = ok1;
         if (tid < 8) sm.dg[tid] = make_float2(sm.Hf[(2 * tid) * 17], sm.Hf[(2 * tid + 1) * 17]);
         __syncthreads();
-        float base = 0.0f;
-        for (int q = 0; q < 4; ++q)
-            if (sm.pd[q]) base = 0.2f * (float)(q + 1) - 0.1f;
-        const bool any1 = sm.pd[0] != 0;
-        const float mu2 = base + 0.05f * (float)(warp + 1);          // refine above the best shift
-        const bool ok2 = any1 && shifted_pd(sm.Hf, sm.Cw[warp], sm.lcolw[warp], mu2, lane);
-        if (lane == 0) sm.pd[4 + warp] = ok2;
+        float lo = 0.0f;
+        for (int q = 0; q < 8; ++q)
+            if (sm.pd[q]) lo = fmaxf(lo, 0.04f + 0.12f * (float)q);
+        const float step = (lo > 0.0f ? 0.12f : 0.04f) * (1.0f / 9.0f);
+        const float mu2 = lo + step * (float)(slot + 1);
+        const bool ok2 = psd_rows && shifted_pd(crow, mu2, i);
+        if (i == 0) sm.pd[8 + slot] = ok2;
         __syncthreads();
-        float best = any1 ? base : 0.0f;
-        for (int q = 0; q < 4; ++q)
-            if (sm.pd[4 + q]) best = fmaxf(best, base + 0.05f * (float)(q + 1));
-        if (tid == 0) sm.mu = best > 0.0f ? best - 6.1035156e-5f : 0.0f;  // - 2^-14
+        float best = lo;
+        for (int q = 0; q < 8; ++q)
+            if (sm.pd[8 + q]) best = fmaxf(best, lo + step * (float)(q + 1));
+        if (tid == 0) sm.mu = best >= 0.00390625f ? best - 6.1035156e-5f : 0.0f;  // - 2^-14
     }
 
-    // Rows are walked in the order of their smallest non-zero |w|: a candidate
-    // saturates every weight of a block exactly when that minimum exceeds 5 s_c,
-    // so after sorting the 32 rows of a warp mostly agree on which candidates
-    // saturate (closed form) and the warp skips the full form together.
+    // Rows are walked in the order of their largest |w|: it fixes where each
+    // class's walk starts (the max-scaling step) and, with it, which candidates
+    // the bounds can exclude, so after sorting the 32 rows of a warp mostly
+    // agree on where to start, what to skip and when to stop.
     const int64_t tile0 = (int64_t)blockIdx.x * kTileRows;
     // counting sort of the tile's rows by a 9-bit key (exponent and first
-    // mantissa bit of the smallest non-zero |w|; rows past c_out last)
+    // mantissa bit of the largest |w|; rows past c_out last)
     for (int i = tid; i < kSortBuckets; i += kThreads) sm.hist[i] = 0;
     __syncthreads();
     uint32_t kb[kRowsPerThread];
@@ -315,10 +309,10 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         if (r < c_out) {
             float wk[16];
             load_block<T>(W + m * mat_stride + r * ld + 16 * j, wk);
-            float mn = __int_as_float(0x7F800000);
+            float mx = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) mn = (wk[i] != 0.0f) ? fminf(mn, fabsf(wk[i])) : mn;
-            key = __float_as_uint(mn);
+            for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(wk[i]));
+            key = __float_as_uint(mx);
         }
         kb[q] = (key == 0xFFFFFFFFu) ? (uint32_t)(kSortBuckets - 1) : min(key >> 22, (uint32_t)(kSortBuckets - 2));
         sm.key[p] = ((unsigned long long)key << 32) | (unsigned)p;
@@ -427,7 +421,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 tail_corr = (sw.x + sw.y) * (sm.mu * 9.5367432e-7f);  // 2^-20 mu
             }
             // the reciprocal-based quotient needs every non-zero |w| >= 2^-100
-            const bool tiny_w = __uint_as_float((uint32_t)(sm.order[rr * kThreads + tid] >> 32)) < 7.888609e-31f;
+            bool tiny_w = false;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tiny_w |= (w[i] != 0.0f) && (fabsf(w[i]) < 7.888609e-31f);
 
 #pragma unroll 1
             for (int f = 0; f < 8; ++f) {
@@ -583,18 +579,21 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 auto below_excluded = [&](int k1) -> bool {
                     if (!rel) return false;
                     const float thr = best_e * up_fac;
-                    const float c3 = __int_as_float(((128 + k1) << 23) | 0x400000);   // 3 * 2^k1
-                    const float c3m = __int_as_float(((128 + k1) << 23) | 0x400002);  // |u| above it: |w| / s0 above 3 * 2^k1
-                    float acc0 = 0.0f, acc1 = 0.0f;
+                    const float nc3 = -__int_as_float(((128 + k1) << 23) | 0x400000);  // -3 * 2^k1
+                    float2 acc = make_float2(0.0f, 0.0f), acc2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const float2 dg = sm.dg[p];
-                        const float d0 = fabsf(u[p].x) > c3m ? __fmaf_rn(-c3, s0, fabsf(w2[p].x)) : 0.0f;  // one rounding
-                        const float d1 = fabsf(u[p].y) > c3m ? __fmaf_rn(-c3, s0, fabsf(w2[p].y)) : 0.0f;
-                        acc0 = __fmaf_rn(d0 * d0, dg.x, acc0);
-                        acc1 = __fmaf_rn(d1 * d1, dg.y, acc1);
+                    for (int p = 0; p < 8; p += 2) {
+                        const float4 d4 = lds128(&sm.dg[p]);
+                        // max(|w| - 3 * 2^k1 s0, 0), one rounding: zero exactly when |w| <= 3 * 2^k1 s0
+                        const float2 d0 = make_float2(fmaxf(__fmaf_rn(nc3, s0, fabsf(w2[p].x)), 0.0f),
+                                                      fmaxf(__fmaf_rn(nc3, s0, fabsf(w2[p].y)), 0.0f));
+                        const float2 d1 = make_float2(fmaxf(__fmaf_rn(nc3, s0, fabsf(w2[p + 1].x)), 0.0f),
+                                                      fmaxf(__fmaf_rn(nc3, s0, fabsf(w2[p + 1].y)), 0.0f));
+                        acc = __ffma2_rn(__fmul2_rn(d0, d0), make_float2(d4.x, d4.y), acc);
+                        acc2 = __ffma2_rn(__fmul2_rn(d1, d1), make_float2(d4.z, d4.w), acc2);
                     }
-                    return __all_sync(0xFFFFFFFFu, (acc0 + acc1) * mu_lb > thr);
+                    acc = __fadd2_rn(acc, acc2);
+                    return __all_sync(0xFFFFFFFFu, (acc.x + acc.y) * mu_lb > thr);
                 };
                 // start at the warp's mean max-scaling index (6 * 2^k >= max |u|)
                 int kst = 0;
