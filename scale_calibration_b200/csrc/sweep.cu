@@ -144,6 +144,7 @@ struct SweepShared {
     float2 dg[8];           // diagonal of H, pairs (for the lower bound)
     int pd[16];             // results of the shifted positive-definiteness tests
     float mu;               // mu <= lambda_min(D^-1/2 H D^-1/2), D = diag(H); 0 disables pruning
+    int next_chunk;         // next 32-row chunk of the sorted order to hand to a warp
 };
 
 // Is C - mu I positive definite? FP32 Cholesky by one half-warp, in registers:
@@ -299,6 +300,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
     // counting sort of the tile's rows by a 9-bit key (exponent and first
     // mantissa bit of the largest |w|; rows past c_out last)
     for (int i = tid; i < kSortBuckets; i += kThreads) sm.hist[i] = 0;
+    if (tid == 0) sm.next_chunk = 0;
     __syncthreads();
     uint32_t kb[kRowsPerThread];
 #pragma unroll
@@ -361,11 +363,16 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
     // every candidate scale is a normal FP32 number: g * 2^-9 >= 2^-126.
     const bool fast = (g >= 1.2037062e-35f) && (g <= 1.0e30f);  // g >= 2^-116
 
-#pragma unroll 1
-    for (int rr = 0; rr < kRowsPerThread; ++rr) {
-        const int64_t r = tile0 + (int64_t)(sm.order[rr * kThreads + tid] & 0xFFFFFFFFu);
+    for (;;) {
+        // warps take 32-row chunks of the sorted order as they finish the last one
+        int chunk = 0;
+        if (lane == 0) chunk = atomicAdd(&sm.next_chunk, 1);
+        chunk = __shfl_sync(0xFFFFFFFFu, chunk, 0);
+        if (chunk >= kTileRows / 32) break;
+        const int pos = chunk * 32 + lane;
+        const int64_t r = tile0 + (int64_t)(sm.order[pos] & 0xFFFFFFFFu);
         const bool active = r < c_out;
-        if (__all_sync(0xFFFFFFFFu, !active)) break;
+        if (__all_sync(0xFFFFFFFFu, !active)) break;  // rows past c_out sort last: so are all later chunks
         float w[16];
         if (active) load_block<T>(W + m * mat_stride + r * ld + 16 * j, w);
         else {
