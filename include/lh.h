@@ -81,15 +81,18 @@ LH_API lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, int6
  *   H[g][j][a][b] += sum_{t in group g} x[t][16j+a] * x[t][16j+b]
  *
  * X: device bf16 [n_tokens_total, ld_x] (first c_in columns used), token-major.
- * offsets: device int64 [n_groups+1] with the token range of each group (one
- *   per matrix / expert: tokens [offsets[g], offsets[g+1])), or NULL for a
- *   single group of all tokens (n_groups must then be 1). Offsets are clamped
- *   to [0, n_tokens_total] and empty or inverted ranges count as empty.
+ * offsets: device int64 [n_groups+1], non-decreasing, with the token range of
+ *   each group (one per matrix / expert: tokens [offsets[g], offsets[g+1])), or
+ *   NULL for a single group of all tokens (n_groups must then be 1). Offsets
+ *   are clamped to [0, n_tokens_total] and empty or inverted ranges count as
+ *   empty. Decreasing offsets whose ranges overlap by more than the workspace
+ *   bound allows make the call record LH_ERR_INVALID_ARG in the workspace
+ *   (see lh_workspace_status); H is then unspecified.
  * H: device f32 [n_groups][c_in/16][16][16], read and written (H += ...):
  *   accumulation can be split over batches and resumed across calls.
  * workspace: device, at least lh_hessian_workspace_bytes(...) bytes, 256-byte
- *   aligned, owned by the caller; it holds per-chunk partial sums and must not
- *   be shared by calls in flight at the same time.
+ *   aligned, owned by the caller; it holds the chunk table and per-chunk
+ *   partial sums and must not be shared by calls in flight at the same time.
  * Numerics: bf16 products are exact in FP32; tensor-core FP32 accumulation
  *   over at most 128 tokens, then FP64 accumulation and one final rounding.
  * n_tokens_total == 0 is a no-op returning LH_OK.
@@ -100,8 +103,9 @@ LH_API lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int64_t 
                                 int64_t ld_x, const int64_t* offsets, int64_t n_groups, float* H,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
-/* Status a kernel left in `workspace` (LH_OK or LH_ERR_TIMEOUT when a bounded
- * wait inside lh_accumulate_hessian gave up). Synchronises `stream`. */
+/* Status a kernel left in `workspace`: LH_OK, LH_ERR_TIMEOUT when a bounded
+ * wait inside lh_accumulate_hessian gave up, or LH_ERR_INVALID_ARG when its
+ * group offsets overlapped beyond the workspace bound. Synchronises `stream`. */
 LH_API lh_status lh_workspace_status(const void* workspace, void* stream);
 
 /* Diagnostics; the pages have no counterpart. Runs on `stream` the bounded

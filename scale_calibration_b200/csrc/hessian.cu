@@ -203,6 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // set-up above overlaps the kernel before (programmatic launch); X, the chunk table
+    // and the workspace header are read only after it has finished
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
 
     const int64_t n_chunks = p.grouped ? (int64_t)(*p.n_chunks_dev) : (p.n_tok + p.chunk - 1) / p.chunk;
     bool ok = true;
@@ -315,6 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(const __grid_co
         *abort_flag = 1;
         atomicExch(p.err, (int)LH_ERR_TIMEOUT);
     }
+    // the reduction may launch now; it waits for this grid to finish before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
     if (*abort_flag) {
         // let copies and MMAs already issued by this CTA land before leaving
@@ -351,10 +357,11 @@ __global__ void wait_timeout_kernel(int* err, uint64_t timeout_ns, int arrive) {
 // into chunks of `chunk` tokens; kfirst[g] = first chunk of group g.
 __global__ void chunk_table_kernel(const int64_t* __restrict__ offsets, int64_t G, int64_t n_tok, int64_t chunk,
                                    int64_t max_chunks, Chunk* __restrict__ table, int32_t* __restrict__ kfirst,
-                                   int32_t* __restrict__ n_chunks_out) {
+                                   int32_t* __restrict__ n_chunks_out, int* __restrict__ status) {
     __shared__ int64_t scan[1024];
     __shared__ int64_t base_s;
     const int tid = threadIdx.x;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the main kernel may set up meanwhile
     if (tid == 0) base_s = 0;
     __syncthreads();
     for (int64_t g0 = 0; g0 < G; g0 += blockDim.x) {
@@ -393,24 +400,43 @@ __global__ void chunk_table_kernel(const int64_t* __restrict__ offsets, int64_t 
         const int64_t n = min(base_s, max_chunks);
         kfirst[G] = (int32_t)n;
         *n_chunks_out = (int32_t)n;
+        // only overlapping (decreasing) offsets hold more chunks than the bound; the chunks
+        // past it are dropped and the call reports it
+        if (base_s > max_chunks) atomicExch(status, (int)LH_ERR_INVALID_ARG);
     }
 }
 
 // H[g][j][e] = fp32(H[g][j][e] + sum_{k in chunks of g} partial[k][j][e]) in FP64, chunk order.
+// One block per group and 8 block columns: each thread keeps 8 independent sums, so the
+// loads of a chunk are in flight together.
 __global__ void __launch_bounds__(256) hessian_reduce_kernel(const float* __restrict__ partial,
                                                              const int32_t* __restrict__ kfirst, int64_t J,
                                                              int64_t n_chunks_plain, float* __restrict__ H) {
-    const int64_t j = blockIdx.x;
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials of the kernel before
+    const int64_t j0 = (int64_t)blockIdx.x * 8;
     const int64_t g = blockIdx.y;
     const int e = threadIdx.x;
     int64_t k0, k1;
     if (kfirst) { k0 = kfirst[g]; k1 = kfirst[g + 1]; }
     else { k0 = 0; k1 = n_chunks_plain; }
     if (k1 <= k0) return;
-    double s = 0.0;
-    for (int64_t k = k0; k < k1; ++k) s += (double)partial[((size_t)k * J + j) * 256 + e];
-    float* h = H + ((size_t)g * J + j) * 256 + e;
-    *h = (float)((double)*h + s);
+    const int nj = (int)min((int64_t)8, J - j0);
+    float* h = H + ((size_t)g * J + j0) * 256 + e;
+    double hs[8], acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        hs[i] = i < nj ? (double)h[i * 256] : 0.0;
+        acc[i] = 0.0;
+    }
+    for (int64_t k = k0; k < k1; ++k) {
+        const float* src = partial + ((size_t)k * J + j0) * 256 + e;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i < nj) acc[i] += (double)src[i * 256];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (i < nj) h[i * 256] = (float)(hs[i] + acc[i]);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -445,7 +471,9 @@ extern "C" lh_status lh_workspace_status(const void* workspace, void* stream) {
     if (s != LH_OK) return s;
     s = cuda_status(cudaStreamSynchronize(st), "synchronise");
     if (s != LH_OK) return s;
-    if (err != 0) return fail((lh_status)err, "a bounded wait in the Hessian kernel expired");
+    if (err == LH_ERR_TIMEOUT) return fail(LH_ERR_TIMEOUT, "a bounded wait in the Hessian kernel expired");
+    if (err != 0)
+        return fail((lh_status)err, "the group offsets overlap: their ranges hold more tokens than n_tokens_total");
     return LH_OK;
 }
 
@@ -524,7 +552,7 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     if (offsets) {
         chunk_table_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, n_tokens_total, plan.chunk, plan.max_chunks,
                                                reinterpret_cast<Chunk*>(ws + plan.ws.table_off), kfirst,
-                                               reinterpret_cast<int32_t*>(ws + 4));
+                                               reinterpret_cast<int32_t*>(ws + 4), reinterpret_cast<int*>(ws));
         s = cuda_status(cudaGetLastError(), "chunk_table_kernel launch");
         if (s != LH_OK) return s;
     }
@@ -537,14 +565,41 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     });
     if (attr_err != cudaSuccess) return cuda_status(attr_err, "set shared memory size");
     int64_t grid = kp.n_items_max < sms ? kp.n_items_max : sms;
-    hessian_tc_kernel<<<(unsigned)grid, kThreads, smem_bytes, st>>>(tmap, kp);
-    s = cuda_status(cudaGetLastError(), "hessian_tc_kernel launch");
+    {
+        // programmatic launch: the set-up of its blocks overlaps the end of the kernel before
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem_bytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        s = cuda_status(cudaLaunchKernelEx(&cfg, hessian_tc_kernel, tmap, kp), "hessian_tc_kernel launch");
+    }
     if (s != LH_OK) return s;
 
     const int64_t plain_chunks = (n_tokens_total + plan.chunk - 1) / plan.chunk;
-    hessian_reduce_kernel<<<dim3((unsigned)J, (unsigned)n_groups), 256, 0, st>>>(
-        kp.partial, offsets ? kfirst : nullptr, J, plain_chunks, H);
-    return cuda_status(cudaGetLastError(), "hessian_reduce_kernel launch");
+    {
+        // launched as a programmatic dependent of the main kernel: its blocks start while
+        // that kernel drains and wait (griddepcontrol.wait) for its partial sums
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((J + 7) / 8), (unsigned)n_groups);
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const float* part = kp.partial;
+        const int32_t* kf = offsets ? kfirst : nullptr;
+        s = cuda_status(cudaLaunchKernelEx(&cfg, hessian_reduce_kernel, part, kf, J, plain_chunks, H),
+                        "hessian_reduce_kernel launch");
+    }
+    return s;
 }
 
 // ---------------------------------------------------------------------------

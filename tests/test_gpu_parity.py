@@ -57,7 +57,7 @@ def test_tiny_layer_bf16_output(cuda_ok):
     (130, 144, 129, "bf16", 2),    # one token past a stage
     (64, 272, 1000, "bf16", 3),    # c_in not a multiple of 128
     (3, 16, 17, "f32", 4),         # smallest block count, one MMA step plus one row
-    (257, 256, 4096, "bf16", 5),   # several chunks per slab
+    (257, 256, 4096, "bf16", 5),   # many token tiles per slab, split over CTA ranges
 ])
 def test_ragged_layers(cuda_ok, c_out, c_in, n_tok, w_dtype, seed):
     _full_parity(synth.make_layer(c_out, c_in, n_tok, seed=seed, w_dtype=w_dtype, outlier_frac=0.001))
@@ -69,6 +69,40 @@ def test_grouped_experts_with_empty_and_tiny_groups(cuda_ok):
     res = _full_parity(layer)
     assert np.all(res["H"][0] == 0) and np.all(res["H"][4] == 0)
     assert np.all(res["codes"][0] == 1) and np.all(res["codes"][4] == 1)  # H = 0: lowest code
+
+
+def test_hessian_many_ragged_groups(cuda_ok):
+    # 70 groups (three empty) over 16 slabs: CTA ranges start and end inside groups and slabs
+    import scale_calibration_b200 as lh
+    rng = np.random.default_rng(31)
+    counts = rng.integers(0, 300, size=70)
+    counts[[3, 10, 11]] = 0
+    layer = synth.make_layer(8, 2048, int(counts.sum()), seed=31, n_mats=70, counts=counts.tolist())
+    _, X, off = gu.to_device(layer)
+    H = torch.zeros(70, 128, 16, 16, device="cuda")
+    wsb = lh.lh_hessian_workspace_bytes(layer.n_tok, 2048, 70)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    lh.lh_accumulate_hessian(X, lh.LH_BF16, layer.n_tok, 2048, X.stride(0), off, 70, H, ws, wsb)
+    assert lh.lh_workspace_status(ws) == 0
+    Hg = H.cpu().numpy()
+    per, whole, bad = gu.hessian_rel_errors(Hg, oracle.hessian(layer.X, c_in=2048, offsets=layer.offsets))
+    assert per <= gu.HESSIAN_RTOL and whole <= gu.HESSIAN_RTOL and bad == 0, (per, whole, bad)
+    assert np.all(Hg[[3, 10, 11]] == 0)
+
+
+def test_hessian_overlapping_offsets_are_reported(cuda_ok):
+    # two groups over the same 1000 tokens hold more tiles than the workspace bound: the call
+    # stays in bounds and the workspace status says the offsets are invalid
+    import scale_calibration_b200 as lh
+    layer = synth.make_layer(8, 128, 1000, seed=32)
+    _, X, _ = gu.to_device(layer)
+    off = torch.tensor([0, 1000, 0, 1000], dtype=torch.int64, device="cuda")
+    H = torch.zeros(3, 8, 16, 16, device="cuda")
+    wsb = lh.lh_hessian_workspace_bytes(1000, 128, 3)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    lh.lh_accumulate_hessian(X, lh.LH_BF16, 1000, 128, 128, off, 3, H, ws, wsb)
+    assert lh.lh_workspace_status(ws) == 1  # LH_ERR_INVALID_ARG
+    assert "overlap" in lh.lh_last_error_message()
 
 
 def test_sparse_nonnegative_activations(cuda_ok):

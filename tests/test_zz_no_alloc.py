@@ -48,10 +48,11 @@ def test_noalloc_matches_workspace_entry_on_consecutive_calls(cuda_ok):
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
     import scale_calibration_b200 as lh
-    n_tok, c_in = 65536, 32768   # needs far more than 16 MiB of partial sums
-    assert lh.lh_hessian_workspace_bytes(n_tok, c_in, 1) > (16 << 20)
+    n_tok, c_in, n_groups = 4096, 32768, 64   # one partial slot per (slab, group): far more than 16 MiB
+    assert lh.lh_hessian_workspace_bytes(n_tok, c_in, n_groups) > (16 << 20)
     H = torch.zeros(1, dtype=torch.float32, device="cuda")
     X = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
-    s = lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, n_tok, c_in, c_in, None, 1, H, check=False)
+    off = torch.zeros(n_groups + 1, dtype=torch.int64, device="cuda")
+    s = lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, n_tok, c_in, c_in, off, n_groups, H, check=False)
     assert s == LH_ERR_WORKSPACE
     assert "16 MiB" in lh.lh_last_error_message()
