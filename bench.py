@@ -36,6 +36,26 @@ SWEEP_FLOP_PER_BLOCK = 126 * 152 * 2   # 16 dw FMA + 136 symmetric-form FMA per 
 FP32_LANES_PER_SM = 128
 
 
+def profiled_traffic(kernel_src: str, summary: str):
+    """DRAM bytes per launch of a kernel, from the ncu summary committed under
+    profiles/, or None when the kernel's source has changed since the counters
+    were taken (the summary records the SHA-256 of the source it profiled)."""
+    import hashlib
+    import re
+    src = os.path.join(ROOT, kernel_src)
+    prof = os.path.join(ROOT, "profiles", summary)
+    if not (os.path.exists(src) and os.path.exists(prof)):
+        return None
+    text = open(prof).read()
+    m_sha = re.search(r"source sha256: ([0-9a-f]{64})", text)
+    m_b = re.search(r"dram bytes per launch: (\d+)", text)
+    if not (m_sha and m_b):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_sha.group(1):
+        return None
+    return int(m_b.group(1))
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -341,15 +361,20 @@ def run_ours(args):
     sweep_tflops = SWEEP_FLOP_PER_BLOCK * n_blocks / (t_sweep / 1e3) / 1e12
     hess_bytes = 2 * c_in * n_tok
     hess_gbs = hess_bytes / (t_hess / 1e3) / 1e9
+    sweep_traffic = profiled_traffic("scale_calibration_b200/csrc/sweep.cu", "sweep_kernel_attn_proj.md") \
+        if args.config == 1 else None
     roofline = dict(bound="alu", kernel="sweep_kernel", achieved=sweep_tflops, peak=fp32_peak, unit="TFLOP/s",
-                    frac=sweep_tflops / fp32_peak, traffic=None,
+                    frac=sweep_tflops / fp32_peak, traffic=sweep_traffic,
+                    traffic_note="DRAM bytes per launch from the committed ncu summary (null if the kernel changed)",
                     peak_note=f"FP32 CUDA-core peak {sms} SMs x 128 lanes x 2 flop x {peaks['sm_max_mhz']:.0f} MHz",
                     flop_per_block=SWEEP_FLOP_PER_BLOCK)
     if clocks.get("sm_mhz"):
         roofline["frac_at_measured_clock"] = sweep_tflops / (fp32_peak * clocks["sm_mhz"] / peaks["sm_max_mhz"])
     hessian = dict(tokens_per_s=n_tok * ws / (t_hess / 1e3) if t_hess > 0 else None, bound="hbm",
                    achieved=hess_gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=hess_gbs / peaks["hbm_gbs"],
-                   bytes_per_launch=hess_bytes, peak_source=peaks["source"])
+                   bytes_per_launch=hess_bytes, peak_source=peaks["source"],
+                   traffic=profiled_traffic("scale_calibration_b200/csrc/hessian.cu", "hessian_tc_kernel_mlp_down.md")
+                   if args.config == 3 else None)
 
     line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=ws, steps=args.steps, warmup=args.warmup,
                 ms_per_step=1e3 * t_all / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,

@@ -407,20 +407,21 @@ __global__ void chunk_table_kernel(const int64_t* __restrict__ offsets, int64_t 
 }
 
 // H[g][j][e] = fp32(H[g][j][e] + sum_{k in chunks of g} partial[k][j][e]) in FP64, chunk order.
-// One block per group and 8 block columns: each thread keeps 8 independent sums, so the
-// loads of a chunk are in flight together.
+// One block per group and `cols` (8) block columns: each thread keeps 8 independent
+// sums, so the loads of a chunk are in flight together (many groups, few chunks each).
 __global__ void __launch_bounds__(256) hessian_reduce_kernel(const float* __restrict__ partial,
                                                              const int32_t* __restrict__ kfirst, int64_t J,
-                                                             int64_t n_chunks_plain, float* __restrict__ H) {
+                                                             int64_t n_chunks_plain, int cols,
+                                                             float* __restrict__ H) {
     asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials of the kernel before
-    const int64_t j0 = (int64_t)blockIdx.x * 8;
+    const int64_t j0 = (int64_t)blockIdx.x * cols;
     const int64_t g = blockIdx.y;
     const int e = threadIdx.x;
     int64_t k0, k1;
     if (kfirst) { k0 = kfirst[g]; k1 = kfirst[g + 1]; }
     else { k0 = 0; k1 = n_chunks_plain; }
     if (k1 <= k0) return;
-    const int nj = (int)min((int64_t)8, J - j0);
+    const int nj = (int)min((int64_t)cols, J - j0);
     float* h = H + ((size_t)g * J + j0) * 256 + e;
     double hs[8], acc[8];
 #pragma unroll
@@ -437,6 +438,25 @@ __global__ void __launch_bounds__(256) hessian_reduce_kernel(const float* __rest
 #pragma unroll
     for (int i = 0; i < 8; ++i)
         if (i < nj) h[i * 256] = (float)(hs[i] + acc[i]);
+}
+
+
+// The same with one block column per block (one group: enough blocks to fill the GPU).
+__global__ void __launch_bounds__(256) hessian_reduce1_kernel(const float* __restrict__ partial,
+                                                              const int32_t* __restrict__ kfirst, int64_t J,
+                                                              int64_t n_chunks_plain, float* __restrict__ H) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials of the kernel before
+    const int64_t j = blockIdx.x;
+    const int64_t g = blockIdx.y;
+    const int e = threadIdx.x;
+    int64_t k0, k1;
+    if (kfirst) { k0 = kfirst[g]; k1 = kfirst[g + 1]; }
+    else { k0 = 0; k1 = n_chunks_plain; }
+    if (k1 <= k0) return;
+    double s = 0.0;
+    for (int64_t k = k0; k < k1; ++k) s += (double)partial[((size_t)k * J + j) * 256 + e];
+    float* h = H + ((size_t)g * J + j) * 256 + e;
+    *h = (float)((double)*h + s);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -585,8 +605,9 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     {
         // launched as a programmatic dependent of the main kernel: its blocks start while
         // that kernel drains and wait (griddepcontrol.wait) for its partial sums
+        const int cols = (n_groups * ((J + 7) / 8) >= 4 * (int64_t)sms) ? 8 : 1;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)((J + 7) / 8), (unsigned)n_groups);
+        cfg.gridDim = dim3((unsigned)((J + cols - 1) / cols), (unsigned)n_groups);
         cfg.blockDim = dim3(256);
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
@@ -596,7 +617,9 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
         cfg.numAttrs = 1;
         const float* part = kp.partial;
         const int32_t* kf = offsets ? kfirst : nullptr;
-        s = cuda_status(cudaLaunchKernelEx(&cfg, hessian_reduce_kernel, part, kf, J, plain_chunks, H),
+        s = cols == 1 ? cuda_status(cudaLaunchKernelEx(&cfg, hessian_reduce1_kernel, part, kf, J, plain_chunks, H),
+                                    "hessian_reduce1_kernel launch")
+                      : cuda_status(cudaLaunchKernelEx(&cfg, hessian_reduce_kernel, part, kf, J, plain_chunks, cols, H),
                         "hessian_reduce_kernel launch");
     }
     return s;
