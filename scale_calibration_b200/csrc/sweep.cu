@@ -133,7 +133,7 @@ constexpr int kTileRows = kThreads * kRowsPerThread;  // rows of one CTA, walked
 constexpr int kSortBuckets = 512;
 
 struct SweepShared {
-    unsigned long long key[kTileRows];    // (bits of max |w|) << 32 | local row
+    unsigned long long key[kTileRows];    // (bits of the heavy channels' max |w|) << 32 | local row
     unsigned long long order[kTileRows];  // the same, grouped by sort bucket
     uint32_t hist[kSortBuckets];
     double Us[136];                     // H_aa, H_ab + H_ba (a < b) in FP64, packed upper triangle
@@ -255,10 +255,15 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
     // subtracted to cover it. mu = 0 (no pruning) when H has a zero diagonal
     // entry with a non-zero off-diagonal entry in its row or a negative diagonal
     // entry, or when mu would fall below 2^-8.
+    unsigned heavy;  // channels a with H_aa >= max_b H_bb / 10 (bit a)
     {
         const int hl = lane >> 4, i = lane & 15;
         const int slot = 2 * warp + hl;  // 0..7
         const float hii = sm.Hf[i * 17];
+        float dmax = hii;
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) dmax = fmaxf(dmax, __shfl_xor_sync(0xFFFFFFFFu, dmax, off));
+        heavy = __ballot_sync(0xFFFFFFFFu, hii >= 0.1f * dmax) & 0xFFFFu;
         bool psd_rows = hii >= 0.0f;
         if (hii == 0.0f)
             for (int b = 0; b < 16; ++b)
@@ -292,13 +297,15 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         if (tid == 0) sm.mu = best >= 0.00390625f ? best - 6.1035156e-5f : 0.0f;  // - 2^-14
     }
 
-    // Rows are walked in the order of their largest |w|: it fixes where each
-    // class's walk starts (the max-scaling step) and, with it, which candidates
-    // the bounds can exclude, so after sorting the 32 rows of a warp mostly
-    // agree on where to start, what to skip and when to stop.
+    // Rows are walked in the order of their largest |w| over the heavy channels
+    // (H_aa at least a tenth of the largest; all channels when those weights are
+    // zero): the error is dominated by those channels, so their range sets where
+    // the optimum lies; each class's walk starts at its max-scaling step. After
+    // sorting, the 32 rows of a warp mostly agree on where to start, what to skip
+    // and when to stop.
     const int64_t tile0 = (int64_t)blockIdx.x * kTileRows;
     // counting sort of the tile's rows by a 9-bit key (exponent and first
-    // mantissa bit of the largest |w|; rows past c_out last)
+    // mantissa bit of that largest |w|; rows past c_out last)
     for (int i = tid; i < kSortBuckets; i += kThreads) sm.hist[i] = 0;
     if (tid == 0) sm.next_chunk = 0;
     __syncthreads();
@@ -311,10 +318,13 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         if (r < c_out) {
             float wk[16];
             load_block<T>(W + m * mat_stride + r * ld + 16 * j, wk);
-            float mx = 0.0f;
+            float mx = 0.0f, mh = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(wk[i]));
-            key = __float_as_uint(mx);
+            for (int i = 0; i < 16; ++i) {
+                mx = fmaxf(mx, fabsf(wk[i]));
+                mh = ((heavy >> i) & 1u) ? fmaxf(mh, fabsf(wk[i])) : mh;
+            }
+            key = __float_as_uint(mh > 0.0f ? mh : mx);
         }
         kb[q] = (key == 0xFFFFFFFFu) ? (uint32_t)(kSortBuckets - 1) : min(key >> 22, (uint32_t)(kSortBuckets - 2));
         sm.key[p] = ((unsigned long long)key << 32) | (unsigned)p;
@@ -380,6 +390,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             for (int i = 0; i < 16; ++i) w[i] = 0.0f;
         }
 
+        const float hw = active ? __uint_as_float((uint32_t)(sm.order[pos] >> 32)) : 0.0f;  // the sort key
         float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
         int best_fk = -1;  // 32 f + k of the best candidate (class f, step k); the code is formed at the end
         bool flag = !fast;
@@ -515,7 +526,8 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                                                          __uint_as_float(max(ep[2 * p + 1], mlo)));
                             q[p] = __ffma2_rn(M, make_float2(-1.0f, -1.0f), __fadd2_rn(u[p], M));  // exact
                         }
-                        if (__any_sync(0xFFFFFFFFu, umax > lim)) {
+                        const bool sat_any = __any_sync(0xFFFFFFFFu, umax > lim);
+                        if (sat_any) {
 #pragma unroll
                             for (int p = 0; p < 8; ++p) {
                                 q[p].x = fminf(fmaxf(q[p].x, -lim), lim);
@@ -544,24 +556,28 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                             E = __int_as_float(0x7F800000);
                             if (up) {
                                 // Every larger scale of the class, 2^k' s0 with k' > k, has its grid
-                                // points in {0, .5, 1, 1.5, 2, 3, 4, 6, 8, 12, ...} 2^k, so a weight
-                                // with |w| / s0 <= 7 * 2^k stays at least its distance to the grid at
-                                // k, |dw| here, away from it (less 2^-23 |w| for the rounding of u).
-                                // Weights at or past 7 * 2^k count zero.
-                                const float c7 = __int_as_float(((129 + k) << 23) | 0x5FFFFD);  // 7 * 2^k (1 - 2^-22)
+                                // points in U = {0, .5, 1, 1.5, 2, 3, 4, 6, 8, 12, 16, ...} 2^k, so each
+                                // weight stays at least its distance to U away from it at every later
+                                // step. Below 6 * 2^k the nearest point of U is q here; above 4 * 2^k U is
+                                // the grid {1, 1.5} 2^m, to which the unclamped magic-constant rounding
+                                // goes, so |w - q s0| before the saturation clamp is that distance for
+                                // every weight (less 2^-23 |w| for the rounding of u).
                                 float tail = lbraw;
-                                if (!__all_sync(0xFFFFFFFFu, umax < c7)) {
+                                if (sat_any) {
                                     float2 tl2 = make_float2(0.0f, 0.0f);
 #pragma unroll
                                     for (int p = 0; p < 8; p += 2) {
                                         const float4 d4 = lds128(&sm.dg[p]);
-                                        const float2 s0q = __fmul2_rn(dw[p], dw[p]), s1q = __fmul2_rn(dw[p + 1], dw[p + 1]);
-                                        const float2 m0 = make_float2(fabsf(u[p].x) < c7 ? s0q.x : 0.0f,
-                                                                      fabsf(u[p].y) < c7 ? s0q.y : 0.0f);
-                                        const float2 m1 = make_float2(fabsf(u[p + 1].x) < c7 ? s1q.x : 0.0f,
-                                                                      fabsf(u[p + 1].y) < c7 ? s1q.y : 0.0f);
-                                        tl2 = __ffma2_rn(m0, make_float2(d4.x, d4.y), tl2);
-                                        tl2 = __ffma2_rn(m1, make_float2(d4.z, d4.w), tl2);
+                                        float2 du[2];
+#pragma unroll
+                                        for (int h = 0; h < 2; ++h) {
+                                            const float2 M = make_float2(__uint_as_float(max(ep[2 * (p + h)], mlo)),
+                                                                         __uint_as_float(max(ep[2 * (p + h) + 1], mlo)));
+                                            const float2 qu = __ffma2_rn(M, make_float2(-1.0f, -1.0f), __fadd2_rn(u[p + h], M));
+                                            du[h] = __ffma2_rn(qu, ns0, w2[p + h]);
+                                        }
+                                        tl2 = __ffma2_rn(__fmul2_rn(du[0], du[0]), make_float2(d4.x, d4.y), tl2);
+                                        tl2 = __ffma2_rn(__fmul2_rn(du[1], du[1]), make_float2(d4.z, d4.w), tl2);
                                     }
                                     tail = tl2.x + tl2.y;
                                 }
@@ -602,10 +618,10 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     acc = __fadd2_rn(acc, acc2);
                     return __all_sync(0xFFFFFFFFu, (acc.x + acc.y) * mu_lb > thr);
                 };
-                // start at the warp's mean max-scaling index (6 * 2^k >= max |u|)
+                // start at the warp's mean max-scaling index of the heavy channels (6 * 2^k >= hw / s0)
                 int kst = 0;
                 {
-                    const float x = umax * 0.16666667f;
+                    const float x = __fdividef(hw, 6.0f * s0);
                     const int e = (int)((__float_as_uint(x) >> 23) & 0xFF) - 127;
                     kst = (x > 1.0f) ? e + ((__float_as_uint(x) & 0x7FFFFF) ? 1 : 0) : 0;
                     kst = max(0, min(n - 1, kst));
