@@ -179,6 +179,33 @@ LH_API lh_status lh_fake_quant(const void* W, lh_dtype w_dtype, int64_t n_mats, 
                         int64_t ld_w, const float* global_amax, const uint8_t* codes, void* W_out,
                         lh_dtype out_dtype, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Packed NVFP4 export, in the same pass as the fake quantisation. The pages
+ * describe NVFP4 as a two-level scale (E2M1 data, an E4M3 block scale per 16
+ * weights, an FP32 global scale) whose scales are computed once when the
+ * checkpoint is made ("NVIDIA Model Optimizer Local-Hessian ..." sections
+ * "Local-Hessian 是什么" and "仅更好的缩放，零运行时成本"; "GitHub推荐：NVIDIA
+ * Model-Optimizer: NVFP4 + QAD ...", section "值得关注的理由"); they give no bit
+ * layout. Layout here:
+ *   packed[m][r][c/2]   u8: the 4-bit OCP E2M1 code of q for column c (sign bit,
+ *                       2 exponent bits with bias 1, 1 mantissa bit), even c in
+ *                       the low nibble, odd c in the high nibble;
+ *                       q = E2M1_RNE_sat(fp32(w/s)) as in lh_fake_quant (q = +-0
+ *                       with the sign of w when s == 0);
+ *   block_scales[m][r][j] u8: the E4M3 code of the block scale (= codes);
+ *   global_scale[m]     f32: g = fp32(global_amax[m] / 2688).
+ * Decoding gives fp32(e2m1(nibble) * fp32(e4m3(scale byte) * g)), bit for bit
+ * the value lh_fake_quant writes before its output cast.
+ * W: device [n_mats][c_out][ld_w]. codes: device u8 [n_mats][c_out][c_in/16].
+ * packed: device, 16-byte aligned, required. block_scales, global_scale and
+ * W_out (the fake-quantised W as in lh_fake_quant, out_dtype) are optional
+ * (NULL: not written). One read of W serves every output.
+ * ---------------------------------------------------------------------- */
+LH_API lh_status lh_quantize_nvfp4(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                            int64_t ld_w, const float* global_amax, const uint8_t* codes, uint8_t* packed,
+                            uint8_t* block_scales, float* global_scale, void* W_out, lh_dtype out_dtype,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -72,6 +72,8 @@ def _L():
         lib.oracle_fake_quant_f32.argtypes = [P, I64, I64, I64, I64, P, P, P]
         lib.oracle_fake_quant_bf16.restype = None
         lib.oracle_fake_quant_bf16.argtypes = [P, I64, I64, I64, I64, P, P, P]
+        lib.oracle_pack_nvfp4.restype = None
+        lib.oracle_pack_nvfp4.argtypes = [P, I64, I64, I64, I64, P, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -198,6 +200,22 @@ def fake_quant(W: np.ndarray, global_amax, codes: np.ndarray, out_bf16: bool = F
         out = np.zeros(W.shape, np.float32)
         _L().oracle_fake_quant_f32(_p(W), n_mats, c_out, c_in, c_in, _p(ga), _p(cd), _p(out))
     return out[0] if squeeze else out
+
+
+def pack_nvfp4(W: np.ndarray, global_amax, codes: np.ndarray):
+    """Packed NVFP4 of W with the given codes: (packed u8 [n_mats, c_out, c_in/2],
+    block scale bytes u8 [n_mats, c_out, c_in/16], global scale f32 [n_mats])."""
+    W = _c(W, np.float32)
+    if W.ndim == 2:
+        W = W[None]
+    n_mats, c_out, c_in = W.shape
+    ga = _c(np.atleast_1d(global_amax), np.float32)
+    cd = _c(codes, np.uint8).reshape(n_mats, c_out, c_in // 16)
+    packed = np.zeros((n_mats, c_out, c_in // 2), np.uint8)
+    scales = np.zeros((n_mats, c_out, c_in // 16), np.uint8)
+    gs = np.zeros(n_mats, np.float32)
+    _L().oracle_pack_nvfp4(_p(W), n_mats, c_out, c_in, c_in, _p(ga), _p(cd), _p(packed), _p(scales), _p(gs))
+    return packed, scales, gs
 
 
 def errors_for_codes(W: np.ndarray, global_amax, H: np.ndarray, codes: np.ndarray) -> np.ndarray:

@@ -285,4 +285,52 @@ void oracle_fake_quant_bf16(const float* W, int64_t n_mats, int64_t c_out, int64
     }
 }
 
+// ---------------------------------------------------------------------------
+// Packed NVFP4 export (the checkpoint form of the same quantisation; the pages
+// describe NVFP4 as a two-level scale: E2M1 data with an E4M3 block scale on
+// top of the FP32 global scale). Readings (the pages give no bit layout): each
+// weight is the 4-bit OCP E2M1 code of q (1 sign bit, 2 exponent bits with
+// bias 1, 1 mantissa bit; exponent field 0 is subnormal: value m * 0.5), two
+// per byte with the even column in the low nibble; the block scale byte is
+// the E4M3 code; the global scale is g. Decoding gives
+// fp32(e2m1(nibble) * fp32(v(byte) * g)), the fake-quantised value.
+// ---------------------------------------------------------------------------
+static unsigned e2m1_code(float q) {
+    const unsigned sign = std::signbit(q) ? 1u : 0u;
+    const double a = std::fabs((double)q);
+    unsigned e, m;
+    if (a < 1.0) {  // subnormal: 0 or 0.5
+        e = 0;
+        m = (unsigned)(a / 0.5);
+    } else {        // normal: a = 2^(e-1) * (1 + m/2)
+        e = (unsigned)std::floor(std::log2(a)) + 1u;
+        m = (unsigned)((a / std::ldexp(1.0, (int)e - 1) - 1.0) * 2.0);
+    }
+    return (sign << 3) | (e << 1) | m;
+}
+
+void oracle_pack_nvfp4(const float* W, int64_t n_mats, int64_t c_out, int64_t c_in, int64_t ld,
+                       const float* global_amax, const uint8_t* codes, uint8_t* packed, uint8_t* scales,
+                       float* gscale) {
+    const int64_t J = c_in / 16;
+    for (int64_t m = 0; m < n_mats; ++m) {
+        const float g = oracle_global_scale(global_amax[m]);
+        gscale[m] = g;
+        for (int64_t r = 0; r < c_out; ++r) {
+            for (int64_t j = 0; j < J; ++j) scales[(m * c_out + r) * J + j] = codes[(m * c_out + r) * J + j];
+            for (int64_t c = 0; c < c_in; c += 2) {
+                unsigned nib[2];
+                for (int h = 0; h < 2; ++h) {
+                    const int code = codes[(m * c_out + r) * J + (c + h) / 16];
+                    const float s = oracle_candidate_scale(code, g);
+                    const float w = W[(m * c_out + r) * ld + c + h];
+                    const float q = (s == 0.0f) ? 0.0f * w : oracle_e2m1_rne(w / s);
+                    nib[h] = e2m1_code(q);
+                }
+                packed[(m * c_out + r) * (c_in / 2) + c / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+            }
+        }
+    }
+}
+
 }  // extern "C"

@@ -19,7 +19,7 @@ LH_BF16, LH_F32 = 0, 1
 EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
-    "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout",
+    "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout", "lh_quantize_nvfp4",
 ]
 
 
@@ -45,6 +45,7 @@ def _load() -> ctypes.CDLL:
         "lh_debug_wait_timeout": (I32, [P, ctypes.c_size_t, I64, I32, P]),
         "lh_sweep_scales": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P]),
         "lh_fake_quant": (I32, [P, I32, I64, I64, I64, I64, P, P, P, I32, P]),
+        "lh_quantize_nvfp4": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P, P, I32, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -158,4 +159,14 @@ def lh_fake_quant(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, codes, W_o
                            _ptr(W_out), _dtype(out_dtype), _stream(stream))
     if check:
         _check(s, "lh_fake_quant")
+    return s
+
+
+def lh_quantize_nvfp4(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, codes, packed, block_scales=None,
+                      global_scale=None, W_out=None, out_dtype=LH_BF16, stream=None, check=True) -> int:
+    s = _lib.lh_quantize_nvfp4(_ptr(W), _dtype(w_dtype), n_mats, c_out, c_in, ld_w, _ptr(global_amax), _ptr(codes),
+                               _ptr(packed), _ptr(block_scales), _ptr(global_scale), _ptr(W_out),
+                               _dtype(out_dtype), _stream(stream))
+    if check:
+        _check(s, "lh_quantize_nvfp4")
     return s

@@ -57,11 +57,24 @@ struct Vec16<float> {
     }
 };
 
-template <typename Tin, typename Tout>
+// 4-bit OCP E2M1 code of an E2M1 value q (sign bit, then exponent field with
+// bias 1 and the mantissa bit): from the FP32 bits, |q| >= 1 has exponent field
+// (FP32 exponent - 126) and its first mantissa bit; 0.5 is the subnormal 0b001.
+__device__ __forceinline__ uint32_t e2m1_nibble(float q) {
+    const uint32_t b = __float_as_uint(q);
+    const uint32_t a = b & 0x7FFFFFFFu;
+    const uint32_t mag = a >= 0x3F800000u ? ((((a >> 23) - 126u) << 1) | ((a >> 22) & 1u)) : (a != 0u ? 1u : 0u);
+    return ((b >> 31) << 3) | mag;
+}
+
+// kOut: write the fake-quantised W; kPack: write the packed NVFP4 nibbles (two
+// per byte, even column in the low nibble) and the block scale bytes.
+template <typename Tin, typename Tout, bool kOut, bool kPack>
 __global__ void __launch_bounds__(256) fake_quant_kernel(const Tin* __restrict__ W, int64_t c_out, int64_t J,
                                                          int64_t ld, const float* __restrict__ gamax,
                                                          const uint8_t* __restrict__ codes,
-                                                         Tout* __restrict__ out, int64_t n_blocks_total) {
+                                                         Tout* __restrict__ out, uint8_t* __restrict__ packed,
+                                                         uint8_t* __restrict__ scales, int64_t n_blocks_total) {
     const int64_t per_mat = c_out * J;
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks_total;
          b += (int64_t)gridDim.x * blockDim.x) {
@@ -69,16 +82,31 @@ __global__ void __launch_bounds__(256) fake_quant_kernel(const Tin* __restrict__
         const int64_t rj = b - m * per_mat;
         const int64_t r = rj / J, j = rj - r * J;
         const float g = __fdiv_rn(__ldg(gamax + m), 2688.0f);
-        const float s = __fmul_rn(e4m3_value(__ldg(codes + b)), g);
+        const uint8_t code = __ldg(codes + b);
+        const float s = __fmul_rn(e4m3_value(code), g);
         float w[16], o[16];
+        uint32_t nib[16];
         Vec16<Tin>::load(W + (m * c_out + r) * ld + 16 * j, w);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float q = (s != 0.0f) ? e2m1_rne(__fdiv_rn(w[i], s)) : copysignf(0.0f, w[i]);
             o[i] = __fmul_rn(q, s);
+            nib[i] = e2m1_nibble(q);
         }
-        Vec16<Tout>::store(out + (m * c_out + r) * (J * 16) + 16 * j, o);
+        if constexpr (kOut) Vec16<Tout>::store(out + (m * c_out + r) * (J * 16) + 16 * j, o);
+        if constexpr (kPack) {
+            uint32_t word[2] = {0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 16; ++i) word[i >> 3] |= nib[i] << (4 * (i & 7));
+            *reinterpret_cast<uint2*>(packed + (m * c_out + r) * (J * 8) + 8 * j) = make_uint2(word[0], word[1]);
+            if (scales) scales[b] = code;
+        }
     }
+}
+
+__global__ void global_scale_kernel(const float* __restrict__ gamax, float* __restrict__ gs, int64_t n) {
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += (int64_t)gridDim.x * blockDim.x)
+        gs[m] = __fdiv_rn(gamax[m], 2688.0f);
 }
 
 template <typename T>
@@ -124,6 +152,24 @@ __global__ void __launch_bounds__(256) absmax_kernel(const T* __restrict__ W, in
     }
 }
 
+template <bool kOut, bool kPack>
+void launch_fake_quant(const void* W, lh_dtype w_dtype, int64_t c_out, int64_t J, int64_t ld,
+                       const float* gamax, const uint8_t* codes, void* out, lh_dtype out_dtype, uint8_t* packed,
+                       uint8_t* scales, int64_t nb, unsigned grid, cudaStream_t st) {
+    if (w_dtype == LH_BF16 && out_dtype == LH_BF16)
+        fake_quant_kernel<uint16_t, uint16_t, kOut, kPack><<<grid, 256, 0, st>>>(
+            (const uint16_t*)W, c_out, J, ld, gamax, codes, (uint16_t*)out, packed, scales, nb);
+    else if (w_dtype == LH_BF16)
+        fake_quant_kernel<uint16_t, float, kOut, kPack><<<grid, 256, 0, st>>>(
+            (const uint16_t*)W, c_out, J, ld, gamax, codes, (float*)out, packed, scales, nb);
+    else if (out_dtype == LH_BF16)
+        fake_quant_kernel<float, uint16_t, kOut, kPack><<<grid, 256, 0, st>>>(
+            (const float*)W, c_out, J, ld, gamax, codes, (uint16_t*)out, packed, scales, nb);
+    else
+        fake_quant_kernel<float, float, kOut, kPack><<<grid, 256, 0, st>>>(
+            (const float*)W, c_out, J, ld, gamax, codes, (float*)out, packed, scales, nb);
+}
+
 }  // namespace
 }  // namespace lh
 
@@ -149,18 +195,44 @@ extern "C" lh_status lh_fake_quant(const void* W, lh_dtype w_dtype, int64_t n_ma
     if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const unsigned gb = (unsigned)blocks;
-    if (w_dtype == LH_BF16 && out_dtype == LH_BF16)
-        fake_quant_kernel<uint16_t, uint16_t><<<gb, 256, 0, st>>>((const uint16_t*)W, c_out, J, ld_w, global_amax,
-                                                                 codes, (uint16_t*)W_out, nb);
-    else if (w_dtype == LH_BF16)
-        fake_quant_kernel<uint16_t, float><<<gb, 256, 0, st>>>((const uint16_t*)W, c_out, J, ld_w, global_amax,
-                                                              codes, (float*)W_out, nb);
-    else if (out_dtype == LH_BF16)
-        fake_quant_kernel<float, uint16_t><<<gb, 256, 0, st>>>((const float*)W, c_out, J, ld_w, global_amax,
-                                                              codes, (uint16_t*)W_out, nb);
+    launch_fake_quant<true, false>(W, w_dtype, c_out, J, ld_w, global_amax, codes, W_out, out_dtype, nullptr, nullptr,
+                                   nb, gb, st);
+    return cuda_status(cudaGetLastError(), "fake_quant_kernel launch");
+}
+
+extern "C" lh_status lh_quantize_nvfp4(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out,
+                                       int64_t c_in, int64_t ld_w, const float* global_amax, const uint8_t* codes,
+                                       uint8_t* packed, uint8_t* block_scales, float* global_scale, void* W_out,
+                                       lh_dtype out_dtype, void* stream) {
+    using namespace lh;
+    clear_error();
+    if (!valid_dtype(w_dtype) || (W_out && !valid_dtype(out_dtype))) return fail(LH_ERR_UNSUPPORTED, "unknown dtype");
+    if (!W || !global_amax || !codes || !packed) return fail(LH_ERR_INVALID_ARG, "null pointer argument");
+    if (n_mats < 1 || c_out < 0 || c_in < 0) return fail(LH_ERR_INVALID_ARG, "n_mats must be >= 1, sizes >= 0");
+    if (c_in % 16 != 0) return fail(LH_ERR_UNSUPPORTED, "c_in=%lld is not a multiple of 16", (long long)c_in);
+    if (ld_w < c_in) return fail(LH_ERR_INVALID_ARG, "ld_w < c_in");
+    if (!aligned16(W) || (ld_w * elem_bytes(w_dtype)) % 16 != 0 || !aligned16(packed) || (W_out && !aligned16(W_out)))
+        return fail(LH_ERR_ALIGNMENT, "W, packed and W_out must be 16-byte aligned, with 16-byte aligned rows of W");
+    if (W == W_out || W == (const void*)packed) return fail(LH_ERR_INVALID_ARG, "outputs must not alias W");
+    const int64_t J = c_in / 16;
+    const int64_t nb = n_mats * c_out * J;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (global_scale) {
+        global_scale_kernel<<<(unsigned)((n_mats + 255) / 256), 256, 0, st>>>(global_amax, global_scale, n_mats);
+        lh_status s = cuda_status(cudaGetLastError(), "global_scale_kernel launch");
+        if (s != LH_OK) return s;
+    }
+    if (nb == 0) return LH_OK;
+    const int sms = sm_count();
+    if (sms <= 0) return fail(LH_ERR_CUDA, "no CUDA device");
+    int64_t blocks = (nb + 255) / 256;
+    if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+    if (W_out)
+        launch_fake_quant<true, true>(W, w_dtype, c_out, J, ld_w, global_amax, codes, W_out, out_dtype, packed,
+                                      block_scales, nb, (unsigned)blocks, st);
     else
-        fake_quant_kernel<float, float><<<gb, 256, 0, st>>>((const float*)W, c_out, J, ld_w, global_amax, codes,
-                                                           (float*)W_out, nb);
+        launch_fake_quant<false, true>(W, w_dtype, c_out, J, ld_w, global_amax, codes, nullptr, LH_F32, packed,
+                                       block_scales, nb, (unsigned)blocks, st);
     return cuda_status(cudaGetLastError(), "fake_quant_kernel launch");
 }
 

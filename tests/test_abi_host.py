@@ -109,3 +109,15 @@ def test_debug_wait_rejects_bad_arguments():
     assert lh.lh_debug_wait_timeout(FAKE + 16, 256, 1000, 0, 0, check=False) == 3
     assert lh.lh_debug_wait_timeout(FAKE, 256, 0, 0, 0, check=False) == 1
     assert lh.lh_debug_wait_timeout(FAKE, 256, 2000000, 0, 0, check=False) == 1
+
+
+def test_quantize_nvfp4_rejects_bad_arguments():
+    lh = _lh()
+    ok = dict(W=FAKE, w_dtype=lh.LH_BF16, n_mats=1, c_out=8, c_in=32, ld_w=32, global_amax=FAKE, codes=FAKE,
+              packed=FAKE + 4096, block_scales=None, global_scale=None, W_out=None, out_dtype=lh.LH_BF16, stream=0,
+              check=False)
+    for over, want in [(dict(packed=None), 1), (dict(codes=None), 1), (dict(W=None), 1), (dict(c_in=20, ld_w=20), 2),
+                       (dict(packed=FAKE + 4104), 3), (dict(W_out=FAKE + 8200), 3), (dict(packed=FAKE), 1),
+                       (dict(W_out=FAKE), 1), (dict(w_dtype=5), 2), (dict(W_out=FAKE + 8192, out_dtype=9), 2)]:
+        assert lh.lh_quantize_nvfp4(**dict(ok, **over)) == want, over
+        assert lh.lh_last_error_message() != ""

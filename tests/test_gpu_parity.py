@@ -105,6 +105,43 @@ def test_hessian_overlapping_offsets_are_reported(cuda_ok):
     assert "overlap" in lh.lh_last_error_message()
 
 
+def _packed_parity(layer, out_dtype):
+    import scale_calibration_b200 as lh
+    W, X, off = gu.to_device(layer)
+    res = gu.run_library(layer, W=W, X=X, off=off, out_dtype=out_dtype)
+    n_mats, c_out, c_in = W.shape
+    codes = torch.from_numpy(res["codes"]).cuda()
+    amax = torch.from_numpy(res["amax"]).cuda()
+    packed = torch.empty(n_mats, c_out, c_in // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(n_mats, c_out, c_in // 16, dtype=torch.uint8, device="cuda")
+    gs = torch.empty(n_mats, dtype=torch.float32, device="cuda")
+    Wq = torch.empty(n_mats, c_out, c_in, dtype=out_dtype, device="cuda")
+    dt = lh.LH_BF16 if out_dtype == torch.bfloat16 else lh.LH_F32
+    lh.lh_quantize_nvfp4(W, W, n_mats, c_out, c_in, W.stride(1), amax, codes, packed, scales, gs, Wq, dt)
+    torch.cuda.synchronize()
+    p_ref, s_ref, g_ref = oracle.pack_nvfp4(layer.W_f32(), res["amax"], res["codes"])
+    assert np.array_equal(packed.cpu().numpy(), p_ref)
+    assert np.array_equal(scales.cpu().numpy(), s_ref)
+    assert np.array_equal(gs.cpu().numpy(), g_ref)
+    wq = Wq.view(torch.int16).cpu().numpy().view(np.uint16) if out_dtype == torch.bfloat16 else Wq.cpu().numpy()
+    assert np.array_equal(wq, res["Wq"])  # the fused pass writes what lh_fake_quant writes
+    # packed only: no optional outputs
+    packed2 = torch.zeros_like(packed)
+    lh.lh_quantize_nvfp4(W, W, n_mats, c_out, c_in, W.stride(1), amax, codes, packed2)
+    torch.cuda.synchronize()
+    assert torch.equal(packed2, packed)
+
+
+def test_packed_nvfp4_export_tiny(cuda_ok):
+    _packed_parity(synth.make_config(0), torch.float32)
+
+
+def test_packed_nvfp4_export_ragged_and_grouped(cuda_ok):
+    _packed_parity(synth.make_layer(130, 144, 129, seed=2, w_dtype="bf16", outlier_frac=0.001), torch.bfloat16)
+    counts = [0, 5, 1, 300, 0, 17, 129, 2100]
+    _packed_parity(synth.make_layer(96, 128, sum(counts), seed=6, n_mats=len(counts), counts=counts), torch.bfloat16)
+
+
 def test_sparse_nonnegative_activations(cuda_ok):
     _full_parity(synth.make_layer(128, 256, 777, seed=7, sparse=0.6))
 
