@@ -161,7 +161,8 @@ LH_API lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, 
  * proven bound on the FP32 rounding error are re-evaluated in FP64, so the
  * chosen code is the exact argmin up to FP64 rounding.
  * W: device bf16 or f32 [n_mats][c_out][ld_w]. global_amax: device f32 [n_mats].
- * H: device f32 [n_mats][c_in/16][16][16] (symmetric; the upper triangle is read).
+ * H: device f32 [n_mats][c_in/16][16][16] (symmetric; the upper triangle is read), or NULL
+ *   for the identity (the weight-MSE sweep of the pages' MSE baseline).
  * best_amax: device f32 [n_mats][c_out][c_in/16]. best_code: device u8, same shape.
  * ---------------------------------------------------------------------- */
 LH_API lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
@@ -205,6 +206,27 @@ LH_API lh_status lh_quantize_nvfp4(const void* W, lh_dtype w_dtype, int64_t n_ma
                             int64_t ld_w, const float* global_amax, const uint8_t* codes, uint8_t* packed,
                             uint8_t* block_scales, float* global_scale, void* W_out, lh_dtype out_dtype,
                             void* stream);
+
+/* ------------------------------------------------------------------------
+ * Baseline block scalers the pages compare Local-Hessian with ("NVIDIA Model
+ * Optimizer Local-Hessian ..." section "Local-Hessian 是什么": max scaling
+ * from the block's largest |w|, four-over-six choosing one of two candidate
+ * scales by the in-block error, and the MSE sweep of all 126 codes on the
+ * weight error). The pages give no formulas; with g = fp32(global_amax/2688):
+ *   LH_SCALE_MAX:           code = E4M3_RNE_sat(fp32(fp32(amax_b / 6) / g)),
+ *                           at least 1 (code 1 when g == 0);
+ *   LH_SCALE_FOUR_OVER_SIX: the codes of amax_b / 6 and amax_b / 4 the same
+ *                           way; the one with the smaller FP64 sum of dw^2 over
+ *                           the block is kept (the lower code on ties);
+ *   LH_SCALE_MSE:           lh_sweep_scales with H = NULL (the identity).
+ * Outputs as lh_sweep_scales: best_code u8 and best_amax = fp32(6 * s_code),
+ * [n_mats][c_out][c_in/16]. W: device bf16 or f32 [n_mats][c_out][ld_w].
+ * ---------------------------------------------------------------------- */
+typedef enum { LH_SCALE_MAX = 0, LH_SCALE_FOUR_OVER_SIX = 1, LH_SCALE_MSE = 2 } lh_scaler;
+
+LH_API lh_status lh_baseline_scales(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                             int64_t ld_w, const float* global_amax, lh_scaler method, float* best_amax,
+                             uint8_t* best_code, void* stream);
 
 #ifdef __cplusplus
 }

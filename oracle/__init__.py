@@ -74,6 +74,10 @@ def _L():
         lib.oracle_fake_quant_bf16.argtypes = [P, I64, I64, I64, I64, P, P, P]
         lib.oracle_pack_nvfp4.restype = None
         lib.oracle_pack_nvfp4.argtypes = [P, I64, I64, I64, I64, P, P, P, P, P]
+        lib.oracle_e4m3_rne.restype = ctypes.c_int
+        lib.oracle_e4m3_rne.argtypes = [F]
+        lib.oracle_baseline_scales.restype = None
+        lib.oracle_baseline_scales.argtypes = [P, I64, I64, I64, I64, P, ctypes.c_int, P, P]
         _lib = lib
     return _lib
 
@@ -200,6 +204,28 @@ def fake_quant(W: np.ndarray, global_amax, codes: np.ndarray, out_bf16: bool = F
         out = np.zeros(W.shape, np.float32)
         _L().oracle_fake_quant_f32(_p(W), n_mats, c_out, c_in, c_in, _p(ga), _p(cd), _p(out))
     return out[0] if squeeze else out
+
+
+def e4m3_rne(x: float) -> int:
+    """E4M3 code of x >= 0, round to nearest even, saturating at 448."""
+    return int(_L().oracle_e4m3_rne(float(x)))
+
+
+BASELINE_MAX, BASELINE_FOUR_OVER_SIX = 0, 1
+
+
+def baseline_scales(W: np.ndarray, global_amax, method: int):
+    """Max scaling (method 0) or four-over-six (method 1): (codes u8, amax f32)
+    of shape [n_mats, c_out, c_in/16]. The MSE baseline is sweep() with H = I."""
+    W = _c(W, np.float32)
+    if W.ndim == 2:
+        W = W[None]
+    n_mats, c_out, c_in = W.shape
+    ga = _c(np.atleast_1d(global_amax), np.float32)
+    code = np.zeros((n_mats, c_out, c_in // 16), np.uint8)
+    amax = np.zeros((n_mats, c_out, c_in // 16), np.float32)
+    _L().oracle_baseline_scales(_p(W), n_mats, c_out, c_in, c_in, _p(ga), int(method), _p(code), _p(amax))
+    return code, amax
 
 
 def pack_nvfp4(W: np.ndarray, global_amax, codes: np.ndarray):

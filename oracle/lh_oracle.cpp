@@ -333,4 +333,72 @@ void oracle_pack_nvfp4(const float* W, int64_t n_mats, int64_t c_out, int64_t c_
     }
 }
 
+// ---------------------------------------------------------------------------
+// Baseline block scalers ([LH] "Local-Hessian 是什么": max scaling takes the
+// block scale from the largest |w| of the 16 weights so they fall inside the
+// E2M1 range; the MSE method sweeps all 126 codes on the weight error; the
+// four-over-six method picks one of two candidate scales by the in-block
+// error). Readings (the pages give no formulas):
+//   max:          code = E4M3_RNE_sat(fp32(fp32(amax_b / 6) / g)), at least 1;
+//   four-over-six: the codes of amax_b / 6 and amax_b / 4 the same way; keep the
+//                 one with the smaller sum of dw^2 (FP64), the lower code on ties;
+//   MSE:          the 126-code sweep with H = I (oracle_sweep with identity H).
+// ---------------------------------------------------------------------------
+
+// E4M3 code of x >= 0, round to nearest (ties to the even code), saturating at
+// 448 (0x7E); written as a search over the 127 non-negative finite codes.
+int oracle_e4m3_rne(float x) {
+    const double v = (double)x;
+    if (!(v > 0.0)) return 0;
+    if (v >= 448.0) return 0x7E;
+    int best = 0;
+    double bd = std::fabs(v - oracle_e4m3_value(0));
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double d = std::fabs(v - oracle_e4m3_value(c));
+        if (d < bd || (d == bd && (c & 1) == 0)) { bd = d; best = c; }
+    }
+    return best;
+}
+
+static double weight_error(const float* w, float g, int code) {
+    const float s = oracle_candidate_scale(code, g);
+    double e = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        const float q = (s != 0.0f) ? oracle_e2m1_rne(w[i] / s) : 0.0f;
+        const double d = (double)q * (double)s - (double)w[i];
+        e += d * d;
+    }
+    return e;
+}
+
+// method 0: max scaling; 1: four-over-six.
+void oracle_baseline_scales(const float* W, int64_t n_mats, int64_t c_out, int64_t c_in, int64_t ld,
+                            const float* global_amax, int method, uint8_t* code_out, float* amax_out) {
+    const int64_t J = c_in / 16;
+    for (int64_t m = 0; m < n_mats; ++m) {
+        const float g = oracle_global_scale(global_amax[m]);
+        for (int64_t r = 0; r < c_out; ++r)
+            for (int64_t j = 0; j < J; ++j) {
+                const float* w = W + (m * c_out + r) * ld + 16 * j;
+                float a = 0.0f;
+                for (int i = 0; i < 16; ++i) a = std::fmax(a, std::fabs(w[i]));
+                auto code_for = [&](float d) {
+                    if (g == 0.0f) return 1;  // every scale is 0
+                    const int c = oracle_e4m3_rne((a / d) / g);
+                    return c < 1 ? 1 : c;
+                };
+                int c = code_for(6.0f);
+                if (method == 1) {
+                    const int c4 = code_for(4.0f);
+                    if (c4 != c) {
+                        const double e6 = weight_error(w, g, c), e4 = weight_error(w, g, c4);
+                        if (e4 < e6 || (e4 == e6 && c4 < c)) c = c4;
+                    }
+                }
+                code_out[(m * c_out + r) * J + j] = (uint8_t)c;
+                amax_out[(m * c_out + r) * J + j] = 6.0f * oracle_candidate_scale(c, g);
+            }
+    }
+}
+
 }  // extern "C"

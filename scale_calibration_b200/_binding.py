@@ -19,8 +19,9 @@ LH_BF16, LH_F32 = 0, 1
 EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
-    "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout", "lh_quantize_nvfp4",
+    "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout", "lh_quantize_nvfp4", "lh_baseline_scales",
 ]
+LH_SCALE_MAX, LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE = range(3)
 
 
 class LHError(RuntimeError):
@@ -46,6 +47,7 @@ def _load() -> ctypes.CDLL:
         "lh_sweep_scales": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P]),
         "lh_fake_quant": (I32, [P, I32, I64, I64, I64, I64, P, P, P, I32, P]),
         "lh_quantize_nvfp4": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P, P, I32, P]),
+        "lh_baseline_scales": (I32, [P, I32, I64, I64, I64, I64, P, I32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -169,4 +171,13 @@ def lh_quantize_nvfp4(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, codes,
                                _dtype(out_dtype), _stream(stream))
     if check:
         _check(s, "lh_quantize_nvfp4")
+    return s
+
+
+def lh_baseline_scales(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, method, best_amax, best_code, stream=None,
+                       check=True) -> int:
+    s = _lib.lh_baseline_scales(_ptr(W), _dtype(w_dtype), n_mats, c_out, c_in, ld_w, _ptr(global_amax), int(method),
+                                _ptr(best_amax), _ptr(best_code), _stream(stream))
+    if check:
+        _check(s, "lh_baseline_scales")
     return s

@@ -227,8 +227,8 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
     const int64_t j = blockIdx.y;
     const int64_t m = blockIdx.z;
 
-    const float* Hj = H + (m * J + j) * 256;
-    for (int i = tid; i < 256; i += kThreads) sm.Hf[i] = Hj[i];
+    const float* Hj = H ? H + (m * J + j) * 256 : nullptr;  // no H: the identity (the weight-MSE sweep)
+    for (int i = tid; i < 256; i += kThreads) sm.Hf[i] = Hj ? Hj[i] : ((i % 17 == 0) ? 1.0f : 0.0f);
     for (int i = tid; i < kPairSlots; i += kThreads) sm.Up[i] = make_float2(0.0f, 0.0f);
     __syncthreads();
     for (int i = tid; i < 256; i += kThreads) {
@@ -696,8 +696,7 @@ extern "C" lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_
     using namespace lh;
     clear_error();
     if (!valid_dtype(w_dtype)) return fail(LH_ERR_UNSUPPORTED, "w_dtype %d is not LH_BF16 or LH_F32", (int)w_dtype);
-    if (!W || !global_amax || !H || !best_amax || !best_code)
-        return fail(LH_ERR_INVALID_ARG, "null pointer argument");
+    if (!W || !global_amax || !best_amax || !best_code) return fail(LH_ERR_INVALID_ARG, "null pointer argument");
     if (n_mats < 1 || c_out < 0 || c_in < 0) return fail(LH_ERR_INVALID_ARG, "n_mats must be >= 1, sizes >= 0");
     if (c_in % 16 != 0) return fail(LH_ERR_UNSUPPORTED, "c_in=%lld is not a multiple of 16", (long long)c_in);
     if (ld_w < c_in) return fail(LH_ERR_INVALID_ARG, "ld_w=%lld < c_in=%lld", (long long)ld_w, (long long)c_in);

@@ -44,7 +44,7 @@ def test_sweep_rejects_bad_arguments():
     ok = dict(W=FAKE, w_dtype=lh.LH_BF16, n_mats=1, c_out=64, c_in=128, ld_w=128, global_amax=FAKE, H=FAKE,
               best_amax=FAKE, best_code=FAKE, stream=0, check=False)
     cases = [
-        (dict(W=0), 1), (dict(H=0), 1), (dict(best_code=0), 1), (dict(n_mats=0), 1), (dict(c_out=-1), 1),
+        (dict(W=0), 1), (dict(global_amax=0), 1), (dict(best_code=0), 1), (dict(n_mats=0), 1), (dict(c_out=-1), 1),
         (dict(c_in=24, ld_w=24), 2), (dict(ld_w=120), 1), (dict(W=FAKE + 2), 3), (dict(ld_w=132), 3),
         (dict(w_dtype=7), 2), (dict(c_in=16 * 70000, ld_w=16 * 70000), 2),
     ]
@@ -121,3 +121,16 @@ def test_quantize_nvfp4_rejects_bad_arguments():
                        (dict(W_out=FAKE), 1), (dict(w_dtype=5), 2), (dict(W_out=FAKE + 8192, out_dtype=9), 2)]:
         assert lh.lh_quantize_nvfp4(**dict(ok, **over)) == want, over
         assert lh.lh_last_error_message() != ""
+
+
+def test_baseline_scales_reject_bad_arguments():
+    lh = _lh()
+    ok = dict(W=FAKE, w_dtype=lh.LH_BF16, n_mats=1, c_out=64, c_in=128, ld_w=128, global_amax=FAKE,
+              method=lh.LH_SCALE_MAX, best_amax=FAKE, best_code=FAKE, stream=0, check=False)
+    for over, want in [(dict(W=0), 1), (dict(best_code=0), 1), (dict(method=7), 2), (dict(c_in=24, ld_w=24), 2),
+                       (dict(ld_w=120), 1), (dict(W=FAKE + 2), 3), (dict(w_dtype=7), 2),
+                       (dict(method=lh.LH_SCALE_FOUR_OVER_SIX, best_amax=0), 1),
+                       (dict(method=lh.LH_SCALE_MSE, W=0), 1), (dict(method=lh.LH_SCALE_MSE, ld_w=132), 3)]:
+        assert lh.lh_baseline_scales(**dict(ok, **over)) == want, over
+        assert lh.lh_last_error_message() != ""
+    assert lh.lh_baseline_scales(**dict(ok, c_out=0)) == 0
