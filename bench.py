@@ -302,6 +302,40 @@ def run_ours(args):
     ex_bytes = (W.numel() * W.element_size() + 2 * codes.numel() + packed.numel() + Wq.numel() * Wq.element_size()
                 + 8 * n_mats)
 
+    # ---- the pages' baseline scalers on the same layer (context beside the Local-Hessian sweep)
+    bl_codes = torch.empty_like(codes)
+    bl_amax = torch.empty_like(bamax)
+    baselines = {}
+    for name, meth in (("max", lh.LH_SCALE_MAX), ("four_over_six", lh.LH_SCALE_FOUR_OVER_SIX),
+                       ("mse_sweep", lh.LH_SCALE_MSE)):
+        for _ in range(3):
+            lh.lh_baseline_scales(W, W, n_mats, c_out, c_in, ld, amax, meth, bl_amax, bl_codes, s)
+        tb = []
+        for _ in range(max(3, min(args.steps, 10))):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lh.lh_baseline_scales(W, W, n_mats, c_out, c_in, ld, amax, meth, bl_amax, bl_codes, s)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            tb.append(e0.elapsed_time(e1))
+        t_b = float(np.median(tb))
+        baselines[name] = dict(ms=t_b, blocks_per_s=n_mats * c_out * J / (t_b / 1e3))
+    # the amax multiplier search (0.25 + 0.1 k, 38 multipliers) with this layer's H
+    for _ in range(3):
+        lh.lh_search_amax(W, W, n_mats, c_out, c_in, ld, amax, H, bl_amax, bl_codes, stream=s)
+    tb = []
+    for _ in range(max(3, min(args.steps, 10))):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        lh.lh_search_amax(W, W, n_mats, c_out, c_in, ld, amax, H, bl_amax, bl_codes, stream=s)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        tb.append(e0.elapsed_time(e1))
+    t_b = float(np.median(tb))
+    baselines["amax_search_hessian"] = dict(ms=t_b, blocks_per_s=n_mats * c_out * J / (t_b / 1e3))
+
     # ---- end to end through the public API with host buffers: every step copies its
     # inputs from pinned host memory and its results (codes, best amax, W_q) back.
     # Consecutive steps are pipelined over two device buffer sets on three streams
@@ -403,6 +437,7 @@ def run_ours(args):
                 config=dict(workload=workload_desc(layer), blocks=n_blocks, tokens=n_tok, l2="flushed",
                             parallelism=f"{ws} independent layers, no collective"),
                 kernels_ms=dict(absmax=t_abs, hessian=t_hess, sweep=t_sweep, fake_quant=t_fq),
+                baseline_scalers=baselines,
                 nvfp4_export=dict(ms=t_ex, bytes_per_launch=int(ex_bytes), bound="hbm",
                                   achieved=ex_bytes / (t_ex / 1e3) / 1e9, unit="GB/s",
                                   frac=ex_bytes / (t_ex / 1e3) / 1e9 / load_peaks()["hbm_gbs"],

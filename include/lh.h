@@ -228,6 +228,24 @@ LH_API lh_status lh_baseline_scales(const void* W, lh_dtype w_dtype, int64_t n_m
                              int64_t ld_w, const float* global_amax, lh_scaler method, float* best_amax,
                              uint8_t* best_code, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Amax multiplier search with the Hessian metric: the calibration's other
+ * weight search ("NVIDIA Model Optimizer Local-Hessian ..." section
+ * "入口 API 与校准流程": step_size 0.1, start_multiplier 0.25,
+ * stop_multiplier 4.0 search the block amax when the FP8 scale sweep is off).
+ * Readings: multipliers m_k = fp32(start + step * k) for k < n_mult (the pages'
+ * values give start 0.25, step 0.1, n_mult 38: the stop is excluded); candidate
+ * k of block b is the max-scaling code of the amax m_k * amax_b,
+ *   code_k = E4M3_RNE_sat(fp32(fp32(fp32(m_k * amax_b) / 6) / g)), at least 1,
+ * and the block keeps the candidate code with the smallest dw^T H dw (the
+ * lowest code on ties), exactly as lh_sweep_scales does over all 126 codes.
+ * Arguments and outputs as lh_sweep_scales (H may be NULL: the identity);
+ * start > 0, step >= 0, 1 <= n_mult <= 4096.
+ * ---------------------------------------------------------------------- */
+LH_API lh_status lh_search_amax(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                         int64_t ld_w, const float* global_amax, const float* H, double start, double step,
+                         int64_t n_mult, float* best_amax, uint8_t* best_code, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,6 +78,9 @@ def _L():
         lib.oracle_e4m3_rne.argtypes = [F]
         lib.oracle_baseline_scales.restype = None
         lib.oracle_baseline_scales.argtypes = [P, I64, I64, I64, I64, P, ctypes.c_int, P, P]
+        D = ctypes.c_double
+        lib.oracle_amax_search.restype = None
+        lib.oracle_amax_search.argtypes = [P, I64, I64, I64, I64, P, P, D, D, I64, P, P, P]
         _lib = lib
     return _lib
 
@@ -226,6 +229,24 @@ def baseline_scales(W: np.ndarray, global_amax, method: int):
     amax = np.zeros((n_mats, c_out, c_in // 16), np.float32)
     _L().oracle_baseline_scales(_p(W), n_mats, c_out, c_in, c_in, _p(ga), int(method), _p(code), _p(amax))
     return code, amax
+
+
+def amax_search(W: np.ndarray, global_amax, H: np.ndarray, start=0.25, step=0.1, n_mult=38):
+    """Amax multiplier search with the Hessian metric: (codes u8, amax f32, err f64)
+    of shape [n_mats, c_out, c_in/16]."""
+    W = _c(W, np.float32)
+    if W.ndim == 2:
+        W = W[None]
+    n_mats, c_out, c_in = W.shape
+    J = c_in // 16
+    ga = _c(np.atleast_1d(global_amax), np.float32)
+    Hd = _c(H, np.float64).reshape(n_mats, J, 16, 16)
+    code = np.zeros((n_mats, c_out, J), np.uint8)
+    amax = np.zeros((n_mats, c_out, J), np.float32)
+    err = np.zeros((n_mats, c_out, J), np.float64)
+    _L().oracle_amax_search(_p(W), n_mats, c_out, c_in, c_in, _p(ga), _p(Hd), float(start), float(step), int(n_mult),
+                            _p(code), _p(amax), _p(err))
+    return code, amax, err
 
 
 def pack_nvfp4(W: np.ndarray, global_amax, codes: np.ndarray):

@@ -401,4 +401,45 @@ void oracle_baseline_scales(const float* W, int64_t n_mats, int64_t c_out, int64
     }
 }
 
+// ---------------------------------------------------------------------------
+// Amax multiplier search ([LH] "入口 API 与校准流程": step_size 0.1,
+// start_multiplier 0.25, stop_multiplier 4.0 are the amax search of the
+// calibration when the FP8 scale sweep is switched off). Reading: multipliers
+// m_k = fp32(start + step * k) for k < n_mult (the stop excluded: 38 values by
+// default); candidate k is the block scale of the amax m_k * amax_b, rounded as
+// in max scaling: code_k = E4M3_RNE_sat(fp32(fp32(fp32(m_k * amax_b) / 6) / g)),
+// at least 1; the block keeps the candidate code with the smallest
+// E = dw^T H dw (FP64, as in the sweep), the lowest code on ties.
+// ---------------------------------------------------------------------------
+void oracle_amax_search(const float* W, int64_t n_mats, int64_t c_out, int64_t c_in, int64_t ld,
+                        const float* global_amax, const double* H, double start, double step, int64_t n_mult,
+                        uint8_t* code_out, float* amax_out, double* err_out) {
+    const int64_t J = c_in / 16;
+    for (int64_t m = 0; m < n_mats; ++m) {
+        const float g = oracle_global_scale(global_amax[m]);
+        for (int64_t r = 0; r < c_out; ++r)
+            for (int64_t j = 0; j < J; ++j) {
+                const float* w = W + (m * c_out + r) * ld + 16 * j;
+                const double* Hj = H + (m * J + j) * 256;
+                float a = 0.0f;
+                for (int i = 0; i < 16; ++i) a = std::fmax(a, std::fabs(w[i]));
+                int best = 0;
+                double be = 0.0;
+                for (int64_t k = 0; k < n_mult; ++k) {
+                    int c = 1;
+                    if (g != 0.0f) {
+                        const float mk = (float)(start + step * (double)k);
+                        c = oracle_e4m3_rne(((mk * a) / 6.0f) / g);
+                        if (c < 1) c = 1;
+                    }
+                    const double e = oracle_candidate_error(w, g, c, Hj);
+                    if (best == 0 || e < be || (e == be && c < best)) { best = c; be = e; }
+                }
+                code_out[(m * c_out + r) * J + j] = (uint8_t)best;
+                amax_out[(m * c_out + r) * J + j] = 6.0f * oracle_candidate_scale(best, g);
+                err_out[(m * c_out + r) * J + j] = be;
+            }
+    }
+}
+
 }  // extern "C"

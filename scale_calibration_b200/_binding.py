@@ -20,6 +20,7 @@ EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
     "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout", "lh_quantize_nvfp4", "lh_baseline_scales",
+    "lh_search_amax",
 ]
 LH_SCALE_MAX, LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE = range(3)
 
@@ -48,6 +49,7 @@ def _load() -> ctypes.CDLL:
         "lh_fake_quant": (I32, [P, I32, I64, I64, I64, I64, P, P, P, I32, P]),
         "lh_quantize_nvfp4": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P, P, I32, P]),
         "lh_baseline_scales": (I32, [P, I32, I64, I64, I64, I64, P, I32, P, P, P]),
+        "lh_search_amax": (I32, [P, I32, I64, I64, I64, I64, P, P, ctypes.c_double, ctypes.c_double, I64, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -180,4 +182,13 @@ def lh_baseline_scales(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, metho
                                 _ptr(best_amax), _ptr(best_code), _stream(stream))
     if check:
         _check(s, "lh_baseline_scales")
+    return s
+
+
+def lh_search_amax(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, H, best_amax, best_code, start=0.25, step=0.1,
+                   n_mult=38, stream=None, check=True) -> int:
+    s = _lib.lh_search_amax(_ptr(W), _dtype(w_dtype), n_mats, c_out, c_in, ld_w, _ptr(global_amax), _ptr(H),
+                            float(start), float(step), int(n_mult), _ptr(best_amax), _ptr(best_code), _stream(stream))
+    if check:
+        _check(s, "lh_search_amax")
     return s

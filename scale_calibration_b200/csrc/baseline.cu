@@ -40,14 +40,6 @@ __device__ __forceinline__ void load16<float>(const float* p, float (&w)[16]) {
     }
 }
 
-// E4M3 code of x >= 0: round to nearest even, saturating at 448 (the hardware
-// conversion; both halves of the pair take x, the low byte is kept).
-__device__ __forceinline__ int e4m3_rne_code(float x) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(x));
-    return r & 0xFF;
-}
-
 // FP64 sum of dw^2 for one candidate, in index order (no contraction).
 __device__ double weight_error(const float (&w)[16], float s) {
     double e = 0.0;

@@ -44,4 +44,12 @@ __device__ __forceinline__ float e2m1_rne(float u) {
     return copysignf(q, u);
 }
 
+// E4M3 code of x >= 0: round to nearest even, saturating at 448 (the hardware
+// conversion; both halves of the pair take x, the low byte is kept).
+__device__ __forceinline__ int e4m3_rne_code(float x) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(x));
+    return r & 0xFF;
+}
+
 }  // namespace lh

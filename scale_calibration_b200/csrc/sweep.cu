@@ -22,6 +22,8 @@
 //    |dw_i| <= |w_i|, so every block whose runner-up is within twice that bound
 //    of the best is re-swept in FP64 by the whole warp. The result is the
 //    exact argmin (up to FP64 rounding), lowest code on ties.
+#include <cmath>
+
 #include "common.cuh"
 #include "quant.cuh"
 
@@ -143,6 +145,7 @@ struct SweepShared {
     float Hf[256];          // H as given, for the FP64 re-sweep
     float2 dg[8];           // diagonal of H, pairs (for the lower bound)
     int pd[16];             // results of the shifted positive-definiteness tests
+    uint32_t allow[4][kThreads];  // amax search: the codes each thread's current block may take
     float mu;               // mu <= lambda_min(D^-1/2 H D^-1/2), D = diag(H); 0 disables pruning
     int next_chunk;         // next 32-row chunk of the sorted order to hand to a warp
 };
@@ -215,11 +218,13 @@ __device__ __forceinline__ float quad_form_smem(const float2 (&dw)[8], const Swe
     return E0 + E1;
 }
 
-template <typename T, bool kURegs>
+// kMask: the amax multiplier search; each block may only take the codes of the
+// amaxes m_k * amax_b, m_k = fp32(m_start + m_step * k), k < n_mult.
+template <typename T, bool kURegs, bool kMask>
 __global__ void __launch_bounds__(kThreads, kURegs ? 2 : 4)
 sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int64_t mat_stride,
              const float* __restrict__ gamax, const float* __restrict__ H, float* __restrict__ best_amax,
-             uint8_t* __restrict__ best_code) {
+             uint8_t* __restrict__ best_code, double m_start, double m_step, int n_mult) {
     __shared__ __align__(16) SweepShared sm;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -391,6 +396,29 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         }
 
         const float hw = active ? __uint_as_float((uint32_t)(sm.order[pos] >> 32)) : 0.0f;  // the sort key
+        if constexpr (kMask) {
+            // the candidate codes of this block: max-scaling codes of m_k * amax_b
+            uint32_t al[4] = {0u, 0u, 0u, 0u};
+            float ab = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ab = fmaxf(ab, fabsf(w[i]));
+            for (int k = 0; k < n_mult; ++k) {
+                int c = 1;
+                if (g != 0.0f) {
+                    const float mk = __double2float_rn(__dadd_rn(m_start, __dmul_rn(m_step, (double)k)));
+                    c = max(1, e4m3_rne_code(__fdiv_rn(__fdiv_rn(__fmul_rn(mk, ab), 6.0f), g)));
+                }
+                al[c >> 5] |= 1u << (c & 31);
+            }
+            __syncwarp();  // the warp's earlier reads of the last block's codes are done
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sm.allow[q][tid] = al[q];
+            __syncwarp();
+        }
+        auto allowed = [&](int code, int t) -> bool {
+            if constexpr (kMask) return (sm.allow[code >> 5][t] >> (code & 31)) & 1u;
+            else return true;
+        };
         float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
         int best_fk = -1;  // 32 f + k of the best candidate (class f, step k); the code is formed at the end
         bool flag = !fast;
@@ -552,7 +580,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         // (only when mu > 0: otherwise E may be negative and nothing is pruned)
                         const float thr = rel ? best_e * up_fac : __int_as_float(0x7F800000);
                         const float lbraw = lb2.x + lb2.y;
-                        if (__all_sync(0xFFFFFFFFu, lbraw * mu_lb > thr)) {
+                        bool out = lbraw * mu_lb > thr;
+                        if constexpr (kMask) out = out || !allowed(class_code(f, x0 + k), tid);
+                        if (__all_sync(0xFFFFFFFFu, out)) {
                             E = __int_as_float(0x7F800000);
                             if (up) {
                                 // Every larger scale of the class, 2^k' s0 with k' > k, has its grid
@@ -586,6 +616,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         } else {
                             E = form(dw);
                         }
+                    }
+                    if constexpr (kMask) {
+                        if (!allowed(class_code(f, x0 + k), tid)) E = __int_as_float(0x7F800000);
                     }
                     if (E < best_e) {
                         second_e = best_e;
@@ -663,7 +696,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             for (int i = 0; i < 16; ++i) wv[i] = __shfl_sync(0xFFFFFFFFu, w[i], src);
             double be = 0.0;
             int bc = 127;
+            const int src_tid = (tid & ~31) + src;
             for (int c = lane + 1; c <= 126; c += 32) {
+                if (!allowed(c, src_tid)) continue;
                 const double e = candidate_error_f64(wv, g, c, sm.Us);
                 if (bc == 127 || e < be) { be = e; bc = c; }
             }
@@ -690,11 +725,12 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 }  // namespace
 }  // namespace lh
 
-extern "C" lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out,
-                                     int64_t c_in, int64_t ld_w, const float* global_amax, const float* H,
-                                     float* best_amax, uint8_t* best_code, void* stream) {
-    using namespace lh;
-    clear_error();
+namespace lh {
+namespace {
+
+lh_status launch_sweep(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in, int64_t ld_w,
+                       const float* global_amax, const float* H, float* best_amax, uint8_t* best_code, bool masked,
+                       double m_start, double m_step, int n_mult, void* stream) {
     if (!valid_dtype(w_dtype)) return fail(LH_ERR_UNSUPPORTED, "w_dtype %d is not LH_BF16 or LH_F32", (int)w_dtype);
     if (!W || !global_amax || !best_amax || !best_code) return fail(LH_ERR_INVALID_ARG, "null pointer argument");
     if (n_mats < 1 || c_out < 0 || c_in < 0) return fail(LH_ERR_INVALID_ARG, "n_mats must be >= 1, sizes >= 0");
@@ -711,11 +747,45 @@ extern "C" lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_
     dim3 grid((unsigned)tiles, (unsigned)J, (unsigned)n_mats);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t mat_stride = c_out * ld_w;
-    if (w_dtype == LH_BF16)
-        sweep_kernel<uint16_t, LH_SWEEP_UREGS><<<grid, kThreads, 0, st>>>(static_cast<const uint16_t*>(W), c_out, J, ld_w,
-                                                          mat_stride, global_amax, H, best_amax, best_code);
-    else
-        sweep_kernel<float, LH_SWEEP_UREGS><<<grid, kThreads, 0, st>>>(static_cast<const float*>(W), c_out, J, ld_w, mat_stride,
-                                                       global_amax, H, best_amax, best_code);
+    if (w_dtype == LH_BF16) {
+        const uint16_t* w = static_cast<const uint16_t*>(W);
+        if (masked)
+            sweep_kernel<uint16_t, false, true><<<grid, kThreads, 0, st>>>(w, c_out, J, ld_w, mat_stride, global_amax, H,
+                                                                          best_amax, best_code, m_start, m_step, n_mult);
+        else
+            sweep_kernel<uint16_t, LH_SWEEP_UREGS, false><<<grid, kThreads, 0, st>>>(
+                w, c_out, J, ld_w, mat_stride, global_amax, H, best_amax, best_code, 0.0, 0.0, 0);
+    } else {
+        const float* w = static_cast<const float*>(W);
+        if (masked)
+            sweep_kernel<float, false, true><<<grid, kThreads, 0, st>>>(w, c_out, J, ld_w, mat_stride, global_amax, H,
+                                                                       best_amax, best_code, m_start, m_step, n_mult);
+        else
+            sweep_kernel<float, LH_SWEEP_UREGS, false><<<grid, kThreads, 0, st>>>(
+                w, c_out, J, ld_w, mat_stride, global_amax, H, best_amax, best_code, 0.0, 0.0, 0);
+    }
     return cuda_status(cudaGetLastError(), "sweep_kernel launch");
+}
+
+}  // namespace
+}  // namespace lh
+
+extern "C" lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out,
+                                     int64_t c_in, int64_t ld_w, const float* global_amax, const float* H,
+                                     float* best_amax, uint8_t* best_code, void* stream) {
+    lh::clear_error();
+    return lh::launch_sweep(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, H, best_amax, best_code, false, 0.0,
+                            0.0, 0, stream);
+}
+
+extern "C" lh_status lh_search_amax(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                                    int64_t ld_w, const float* global_amax, const float* H, double start, double step,
+                                    int64_t n_mult, float* best_amax, uint8_t* best_code, void* stream) {
+    using namespace lh;
+    clear_error();
+    if (!(start > 0.0) || !(step >= 0.0) || !std::isfinite(start) || !std::isfinite(step))
+        return fail(LH_ERR_INVALID_ARG, "start must be > 0 and step >= 0, both finite");
+    if (n_mult < 1 || n_mult > 4096) return fail(LH_ERR_INVALID_ARG, "n_mult must be in [1, 4096]");
+    return launch_sweep(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, H, best_amax, best_code, true, start, step,
+                        (int)n_mult, stream);
 }

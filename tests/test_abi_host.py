@@ -134,3 +134,15 @@ def test_baseline_scales_reject_bad_arguments():
         assert lh.lh_baseline_scales(**dict(ok, **over)) == want, over
         assert lh.lh_last_error_message() != ""
     assert lh.lh_baseline_scales(**dict(ok, c_out=0)) == 0
+
+
+def test_search_amax_rejects_bad_arguments():
+    lh = _lh()
+    ok = dict(W=FAKE, w_dtype=lh.LH_BF16, n_mats=1, c_out=64, c_in=128, ld_w=128, global_amax=FAKE, H=FAKE,
+              best_amax=FAKE, best_code=FAKE, start=0.25, step=0.1, n_mult=38, stream=0, check=False)
+    for over, want in [(dict(W=0), 1), (dict(best_code=0), 1), (dict(start=0.0), 1), (dict(step=-0.1), 1),
+                       (dict(n_mult=0), 1), (dict(n_mult=5000), 1), (dict(start=float("nan")), 1),
+                       (dict(c_in=24, ld_w=24), 2), (dict(W=FAKE + 2), 3), (dict(w_dtype=7), 2)]:
+        assert lh.lh_search_amax(**dict(ok, **over)) == want, over
+        assert lh.lh_last_error_message() != ""
+    assert lh.lh_search_amax(**dict(ok, c_out=0)) == 0
