@@ -465,6 +465,97 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+def run_sharded(args):
+    """One layer split over the ranks (strong scaling): each rank holds a share of
+    the calibration tokens and of the rows; the global amax is a MAX all-reduce,
+    the Hessian a SUM all-reduce of the ranks' partial H (NCCL), and each rank
+    sweeps and fake-quantises its rows with the full H."""
+    import torch
+    import torch.distributed as dist
+    ws, rank, local = dist_setup("nccl")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import scale_calibration_b200 as lh
+    import synth
+    from scale_calibration_b200 import distributed as lhd
+
+    layer = synth.make_config(args.config)
+    n_mats, c_out, c_in, n_tok = layer.n_mats, layer.c_out, layer.c_in, layer.n_tok
+    J = c_in // 16
+    grouped = layer.offsets is not None
+    n_groups = n_mats if grouped else 1
+    t0, t1, loc = lhd.token_shard(n_tok, rank, ws, layer.offsets)
+    r0, r1 = lhd.row_shard(c_out, rank, ws)
+    rows = r1 - r0
+    Wn = layer.W[:, r0:r1]
+    W_host = (torch.from_numpy(np.ascontiguousarray(Wn).view(np.int16)).view(torch.bfloat16) if layer.w_dtype == "bf16"
+              else torch.from_numpy(np.ascontiguousarray(Wn)))
+    X_host = torch.from_numpy(np.ascontiguousarray(layer.X[t0:t1]).view(np.int16)).view(torch.bfloat16)
+    W = W_host.to(dev)
+    X = X_host.to(dev)
+    n_loc = t1 - t0
+    off = torch.from_numpy(loc).to(dev) if grouped else None
+    amax = torch.empty(n_mats, dtype=torch.float32, device=dev)
+    H = torch.zeros(n_groups, J, 16, 16, dtype=torch.float32, device=dev)
+    wsb = lh.lh_hessian_workspace_bytes(max(n_loc, 1), c_in, n_groups)
+    wsp = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    codes = torch.empty(n_mats, rows, J, dtype=torch.uint8, device=dev)
+    bamax = torch.empty(n_mats, rows, J, dtype=torch.float32, device=dev)
+    Wq = torch.empty(n_mats, rows, c_in, dtype=W.dtype, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 1 << 28) // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    ld = W.stride(1)
+
+    def step():
+        H.zero_()
+        lh.lh_absmax(W, W, n_mats, rows, c_in, ld, amax, s)
+        if ws > 1:
+            dist.all_reduce(amax, op=dist.ReduceOp.MAX)
+        if n_loc > 0:
+            lhd.accumulate_hessian_sharded(X, n_loc, c_in, off, n_groups, H, wsp, wsb, s, check_status=False)
+        else:
+            lhd.allreduce_hessian(H)
+        lh.lh_sweep_scales(W, W, n_mats, rows, c_in, ld, amax, H, bamax, codes, s)
+        lh.lh_fake_quant(W, W, n_mats, rows, c_in, ld, amax, codes, Wq, Wq, s)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    assert n_loc == 0 or lh.lh_workspace_status(wsp, s) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    sampler = ClockSampler(dev.index)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for _ in range(args.steps):
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(e0.elapsed_time(e1) / 1e3)
+    clocks = sampler.stop()
+    t_all = max_over_ranks(float(sum(ts)), ws, dev)
+    n_blocks = n_mats * c_out * J
+    value = n_blocks * args.steps / t_all
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=ws, steps=args.steps, warmup=args.warmup,
+                ms_per_step=1e3 * t_all / args.steps, higher_is_better=True, scaling="strong", vs_baseline=None,
+                dtype="f32", data="synthetic",
+                config=dict(workload=workload_desc(layer), blocks=n_blocks, tokens=n_tok, l2="flushed",
+                            parallelism=f"{ws} ranks: tokens and rows sharded, amax MAX and H SUM all-reduce (NCCL)"),
+                gpu_launches=(4 + (1 if grouped else 0) + 1) * args.steps, clocks=clocks)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -474,11 +565,16 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="0 tiny, 1 attn_proj, 2 mlp_up, 3 mlp_down, 4 moe_experts")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--mode", choices=["layers", "sharded"], default="layers",
+                    help="layers: each rank calibrates its own layer (weak scaling); sharded: one layer split over "
+                         "the ranks with an all-reduce of H (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "sharded":
+        run_sharded(args)
     else:
         run_ours(args)
 
