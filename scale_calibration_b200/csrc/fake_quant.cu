@@ -6,6 +6,8 @@
 //
 // Both kernels stream W once from HBM: one thread per 16-weight block
 // (32 or 64 contiguous bytes, 16-byte vector loads and stores).
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "quant.cuh"
 
@@ -57,48 +59,91 @@ struct Vec16<float> {
     }
 };
 
-// 4-bit OCP E2M1 code of an E2M1 value q (sign bit, then exponent field with
-// bias 1 and the mantissa bit): from the FP32 bits, |q| >= 1 has exponent field
-// (FP32 exponent - 126) and its first mantissa bit; 0.5 is the subnormal 0b001.
-__device__ __forceinline__ uint32_t e2m1_nibble(float q) {
-    const uint32_t b = __float_as_uint(q);
-    const uint32_t a = b & 0x7FFFFFFFu;
-    const uint32_t mag = a >= 0x3F800000u ? ((((a >> 23) - 126u) << 1) | ((a >> 22) & 1u)) : (a != 0u ? 1u : 0u);
-    return ((b >> 31) << 3) | mag;
+// Two 4-bit OCP E2M1 codes at once (sign bit, 2 exponent bits with bias 1,
+// 1 mantissa bit): round to nearest even with saturation at +-6, the hardware
+// conversion (its first operand goes to the high nibble); and their exact
+// values back.
+__device__ __forceinline__ uint32_t e2m1x2_codes(float lo, float hi) {
+    uint16_t r;
+    asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u16.u8 %0, t;\n}" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float2 e2m1x2_values(uint32_t codes) {
+    uint32_t h2;
+    asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}" : "=r"(h2) : "r"(codes));
+    const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+    return __half22float2(h);  // .x from the low nibble
 }
 
 // kOut: write the fake-quantised W; kPack: write the packed NVFP4 nibbles (two
 // per byte, even column in the low nibble) and the block scale bytes.
+// One thread per block, the 16 weights in one fused pass (quotient, E2M1
+// rounding, product, packing) so few values stay live and more CTAs fit an SM.
 template <typename Tin, typename Tout, bool kOut, bool kPack>
-__global__ void __launch_bounds__(256) fake_quant_kernel(const Tin* __restrict__ W, int64_t c_out, int64_t J,
-                                                         int64_t ld, const float* __restrict__ gamax,
-                                                         const uint8_t* __restrict__ codes,
-                                                         Tout* __restrict__ out, uint8_t* __restrict__ packed,
-                                                         uint8_t* __restrict__ scales, int64_t n_blocks_total) {
+__global__ void __launch_bounds__(256, 4) fake_quant_kernel(const Tin* __restrict__ W, int64_t c_out, int64_t J,
+                                                            int64_t ld, const float* __restrict__ gamax,
+                                                            const uint8_t* __restrict__ codes,
+                                                            Tout* __restrict__ out, uint8_t* __restrict__ packed,
+                                                            uint8_t* __restrict__ scales, int64_t n_blocks_total) {
     const int64_t per_mat = c_out * J;
+    const bool dense = ld == 16 * J;  // W rows back to back: block b starts at element 16 b
+    int64_t m_cached = -1;
+    float g = 0.0f;
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < n_blocks_total;
          b += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = b / per_mat;
-        const int64_t rj = b - m * per_mat;
-        const int64_t r = rj / J, j = rj - r * J;
-        const float g = __fdiv_rn(__ldg(gamax + m), 2688.0f);
+        int64_t m = 0, src = 16 * b;
+        if (dense) {
+            if (per_mat != n_blocks_total) m = b / per_mat;
+        } else {
+            m = b / per_mat;
+            const int64_t rj = b - m * per_mat;
+            const int64_t r = rj / J, j = rj - r * J;
+            src = (m * c_out + r) * ld + 16 * j;
+        }
+        if (m != m_cached) {
+            g = __fdiv_rn(__ldg(gamax + m), 2688.0f);
+            m_cached = m;
+        }
         const uint8_t code = __ldg(codes + b);
         const float s = __fmul_rn(e4m3_value(code), g);
-        float w[16], o[16];
-        uint32_t nib[16];
-        Vec16<Tin>::load(W + (m * c_out + r) * ld + 16 * j, w);
+        float w[16];
+        Vec16<Tin>::load(W + src, w);
+        // fp32(w / s): from one correctly rounded reciprocal y = RN(1/s), q = RN(w y),
+        // r = w - s q (exact, one FMA), RN(q + r y) is the correctly rounded quotient
+        // (P. Markstein, IBM J. Res. Dev. 34(1), 1990) while s is normal and no
+        // non-zero |w| is below 2^-100; other blocks divide.
+        float mn = __int_as_float(0x7F800000);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float q = (s != 0.0f) ? e2m1_rne(__fdiv_rn(w[i], s)) : copysignf(0.0f, w[i]);
-            o[i] = __fmul_rn(q, s);
-            nib[i] = e2m1_nibble(q);
+        for (int i = 0; i < 16; ++i) mn = (w[i] != 0.0f) ? fminf(mn, fabsf(w[i])) : mn;
+        const bool fast = s >= 1.17549435e-38f && mn >= 7.888609e-31f;
+        const float y = fast ? __frcp_rn(s) : 0.0f;
+        float o[16];
+        uint32_t word[2] = {0u, 0u};
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            float u[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float wi = w[2 * p + h];
+                if (fast) {
+                    const float q0 = __fmul_rn(wi, y);
+                    // the last FMA turns -0 (w = -0) into +0; the quotient's sign is that of w
+                    u[h] = copysignf(__fmaf_rn(__fmaf_rn(-q0, s, wi), y, q0), wi);
+                } else {
+                    u[h] = (s != 0.0f) ? __fdiv_rn(wi, s) : copysignf(0.0f, wi);
+                }
+            }
+            const uint32_t c2 = e2m1x2_codes(u[0], u[1]);  // element 2p in the low nibble
+            if constexpr (kOut) {
+                const float2 q = e2m1x2_values(c2);
+                o[2 * p] = __fmul_rn(q.x, s);
+                o[2 * p + 1] = __fmul_rn(q.y, s);
+            }
+            if constexpr (kPack) word[p >> 2] |= c2 << (8 * (p & 3));
         }
-        if constexpr (kOut) Vec16<Tout>::store(out + (m * c_out + r) * (J * 16) + 16 * j, o);
+        if constexpr (kOut) Vec16<Tout>::store(out + 16 * b, o);
         if constexpr (kPack) {
-            uint32_t word[2] = {0u, 0u};
-#pragma unroll
-            for (int i = 0; i < 16; ++i) word[i >> 3] |= nib[i] << (4 * (i & 7));
-            *reinterpret_cast<uint2*>(packed + (m * c_out + r) * (J * 8) + 8 * j) = make_uint2(word[0], word[1]);
+            *reinterpret_cast<uint2*>(packed + 8 * b) = make_uint2(word[0], word[1]);
             if (scales) scales[b] = code;
         }
     }
@@ -192,7 +237,7 @@ extern "C" lh_status lh_fake_quant(const void* W, lh_dtype w_dtype, int64_t n_ma
     const int sms = sm_count();
     if (sms <= 0) return fail(LH_ERR_CUDA, "no CUDA device");
     int64_t blocks = (nb + 255) / 256;
-    if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+    if (blocks > (int64_t)sms * 32) blocks = (int64_t)sms * 32;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const unsigned gb = (unsigned)blocks;
     launch_fake_quant<true, false>(W, w_dtype, c_out, J, ld_w, global_amax, codes, W_out, out_dtype, nullptr, nullptr,
@@ -226,7 +271,7 @@ extern "C" lh_status lh_quantize_nvfp4(const void* W, lh_dtype w_dtype, int64_t 
     const int sms = sm_count();
     if (sms <= 0) return fail(LH_ERR_CUDA, "no CUDA device");
     int64_t blocks = (nb + 255) / 256;
-    if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+    if (blocks > (int64_t)sms * 32) blocks = (int64_t)sms * 32;
     if (W_out)
         launch_fake_quant<true, true>(W, w_dtype, c_out, J, ld_w, global_amax, codes, W_out, out_dtype, packed,
                                       block_scales, nb, (unsigned)blocks, st);

@@ -142,6 +142,57 @@ def test_packed_nvfp4_export_ragged_and_grouped(cuda_ok):
     _packed_parity(synth.make_layer(96, 128, sum(counts), seed=6, n_mats=len(counts), counts=counts), torch.bfloat16)
 
 
+def test_signed_zero_weights_keep_their_sign(cuda_ok):
+    # -0 weights quantise to -0: W_q and the packed sign bit, compared as bits
+    import scale_calibration_b200 as lh
+    for w_dtype, out_dtype in (("f32", torch.float32), ("bf16", torch.bfloat16)):
+        layer = synth.make_layer(64, 128, 256, seed=51, w_dtype=w_dtype)
+        if w_dtype == "f32":
+            layer.W[0, ::3, ::5] = np.float32(-0.0)
+        else:
+            layer.W[0, ::3, ::5] = np.uint16(0x8000)
+        W, X, off = gu.to_device(layer)
+        res = gu.run_library(layer, W=W, X=X, off=off, out_dtype=out_dtype)
+        n_mats, c_out, c_in = W.shape
+        bf = out_dtype == torch.bfloat16
+        ref = oracle.fake_quant(layer.W_f32(), res["amax"], res["codes"], out_bf16=bf).reshape(res["Wq"].shape)
+        got = res["Wq"]
+        if not bf:
+            ref, got = ref.view(np.uint32), got.view(np.uint32)
+        assert np.array_equal(ref, got)
+        packed = torch.empty(n_mats, c_out, c_in // 2, dtype=torch.uint8, device="cuda")
+        lh.lh_quantize_nvfp4(W, W, n_mats, c_out, c_in, W.stride(1), torch.from_numpy(res["amax"]).cuda(),
+                             torch.from_numpy(res["codes"]).cuda(), packed)
+        torch.cuda.synchronize()
+        p_ref, _, _ = oracle.pack_nvfp4(layer.W_f32(), res["amax"], res["codes"])
+        assert np.array_equal(packed.cpu().numpy(), p_ref)
+
+
+def test_e2m1_ties_and_saturation_through_fake_quant_and_export(cuda_ok):
+    # every E2M1 rounding tie, its FP32 neighbours, grid points, saturation, tiny values and
+    # signed zeros, at four block scales: W_q bits and packed bytes equal the oracle's
+    import scale_calibration_b200 as lh
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1, 1.5, 2, 3, 4, 6, 6.5, 7, 100, 1e-30, 0], np.float32)
+    vals = np.concatenate([ties, np.nextafter(ties, np.float32(0)), np.nextafter(ties, np.float32(1e9))])
+    vals = np.concatenate([vals, -vals, [np.float32(-0.0)]]).astype(np.float32)
+    n = ((len(vals) + 15) // 16) * 16
+    Wn = np.zeros((1, 4, n), np.float32)
+    Wn[0, :, :len(vals)] = vals
+    for r, f in enumerate((1.0, 2.0, 0.5, 1.5)):
+        Wn[0, r] *= np.float32(f)
+    cd = np.repeat(np.array([0x38, 0x40, 0x30, 0x3C], np.uint8)[:, None], n // 16, axis=1)[None]  # s = f (g = 1)
+    amax = np.array([2688.0], np.float32)
+    W, A, C = (torch.from_numpy(a).cuda() for a in (Wn, amax, cd))
+    out = torch.empty_like(W)
+    pk = torch.zeros(1, 4, n // 2, dtype=torch.uint8, device="cuda")
+    lh.lh_fake_quant(W, lh.LH_F32, 1, 4, n, n, A, C, out, lh.LH_F32)
+    lh.lh_quantize_nvfp4(W, lh.LH_F32, 1, 4, n, n, A, C, pk)
+    torch.cuda.synchronize()
+    ref = oracle.fake_quant(Wn, amax, cd).reshape(Wn.shape)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    assert np.array_equal(pk.cpu().numpy(), oracle.pack_nvfp4(Wn, amax, cd)[0])
+
+
 def test_sparse_nonnegative_activations(cuda_ok):
     _full_parity(synth.make_layer(128, 256, 777, seed=7, sparse=0.6))
 
