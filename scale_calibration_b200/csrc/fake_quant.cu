@@ -166,8 +166,8 @@ __global__ void __launch_bounds__(256) absmax_kernel(const T* __restrict__ W, in
     float mx = 0.0f;
     for (int64_t r = (int64_t)blockIdx.x * warps + (threadIdx.x >> 5); r < rows; r += (int64_t)gridDim.x * warps) {
         const T* row = base + r * ld;
-        for (int64_t v = lane; v < nv; v += 32) {
-            const uint4 t = __ldg(reinterpret_cast<const uint4*>(row) + v);
+        const uint4* rv = reinterpret_cast<const uint4*>(row);
+        auto fold = [&](const uint4& t) {
             const uint32_t u[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -178,7 +178,13 @@ __global__ void __launch_bounds__(256) absmax_kernel(const T* __restrict__ W, in
                     mx = fmaxf(mx, fabsf(__uint_as_float(u[i])));
                 }
             }
+        };
+        int64_t v = lane;
+        for (; v + 96 < nv; v += 128) {  // four independent 16-byte loads in flight per lane
+            const uint4 t0 = __ldg(rv + v), t1 = __ldg(rv + v + 32), t2 = __ldg(rv + v + 64), t3 = __ldg(rv + v + 96);
+            fold(t0); fold(t1); fold(t2); fold(t3);
         }
+        for (; v < nv; v += 32) fold(__ldg(rv + v));
         for (int64_t c = nv * V + lane; c < cols; c += 32) {
             const float x = sizeof(T) == 2 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[c])
                                            : reinterpret_cast<const float*>(row)[c];
@@ -193,8 +199,17 @@ __global__ void __launch_bounds__(256) absmax_kernel(const T* __restrict__ W, in
     if (threadIdx.x == 0) {
         float v = 0.0f;
         for (int i = 0; i < warps; ++i) v = fmaxf(v, red[i]);
+        // launched as a programmatic dependent of absmax_init_kernel: the loads above
+        // overlap it, the atomics wait for its zeros
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         atomicMax(out + m, __float_as_uint(v));  // non-negative floats order like their bits
     }
+}
+
+__global__ void absmax_init_kernel(unsigned int* __restrict__ out, int64_t n) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        out[i] = 0u;
 }
 
 template <bool kOut, bool kPack>
@@ -292,7 +307,8 @@ extern "C" lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, 
     if (!aligned16(W) || (ld * elem_bytes(w_dtype)) % 16 != 0)
         return fail(LH_ERR_ALIGNMENT, "W must be 16-byte aligned with 16-byte aligned rows");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    lh_status s = cuda_status(cudaMemsetAsync(out_amax, 0, sizeof(float) * (size_t)n_mats, st), "memset amax");
+    absmax_init_kernel<<<(unsigned)((n_mats + 255) / 256), 256, 0, st>>>((unsigned int*)out_amax, n_mats);
+    lh_status s = cuda_status(cudaGetLastError(), "absmax_init_kernel launch");
     if (s != LH_OK) return s;
     if (rows == 0 || cols == 0) return LH_OK;
     const int sms = sm_count();
@@ -301,10 +317,21 @@ extern "C" lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, 
     int64_t cap = ((int64_t)sms * 8 + n_mats - 1) / n_mats;
     if (cap < 1) cap = 1;
     if (per > cap) per = cap;
-    dim3 grid((unsigned)per, (unsigned)n_mats);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)per, (unsigned)n_mats);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    unsigned int* o = (unsigned int*)out_amax;
     if (w_dtype == LH_BF16)
-        absmax_kernel<uint16_t><<<grid, 256, 0, st>>>((const uint16_t*)W, rows, cols, ld, (unsigned int*)out_amax);
+        s = cuda_status(cudaLaunchKernelEx(&cfg, absmax_kernel<uint16_t>, (const uint16_t*)W, rows, cols, ld, o),
+                        "absmax_kernel launch");
     else
-        absmax_kernel<float><<<grid, 256, 0, st>>>((const float*)W, rows, cols, ld, (unsigned int*)out_amax);
-    return cuda_status(cudaGetLastError(), "absmax_kernel launch");
+        s = cuda_status(cudaLaunchKernelEx(&cfg, absmax_kernel<float>, (const float*)W, rows, cols, ld, o),
+                        "absmax_kernel launch");
+    return s;
 }
