@@ -6,74 +6,10 @@
 //
 // Both kernels stream W once from HBM: one thread per 16-weight block
 // (32 or 64 contiguous bytes, 16-byte vector loads and stores).
-#include <cuda_fp16.h>
-
-#include "common.cuh"
-#include "quant.cuh"
+#include "nvfp4_block.cuh"
 
 namespace lh {
 namespace {
-
-template <typename T>
-struct Vec16;
-
-template <>
-struct Vec16<uint16_t> {
-    __device__ static void load(const uint16_t* p, float (&w)[16]) {
-        const uint4* q = reinterpret_cast<const uint4*>(p);
-        const uint4 a = __ldg(q), b = __ldg(q + 1);
-        const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            w[2 * i] = __uint_as_float(v[i] << 16);
-            w[2 * i + 1] = __uint_as_float(v[i] & 0xFFFF0000u);
-        }
-    }
-    __device__ static void store(uint16_t* p, const float (&o)[16]) {
-        uint32_t v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);  // RNE
-            v[i] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        uint4* q = reinterpret_cast<uint4*>(p);
-        q[0] = make_uint4(v[0], v[1], v[2], v[3]);
-        q[1] = make_uint4(v[4], v[5], v[6], v[7]);
-    }
-};
-
-template <>
-struct Vec16<float> {
-    __device__ static void load(const float* p, float (&w)[16]) {
-        const float4* q = reinterpret_cast<const float4*>(p);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float4 t = __ldg(q + i);
-            w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
-        }
-    }
-    __device__ static void store(float* p, const float (&o)[16]) {
-        float4* q = reinterpret_cast<float4*>(p);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) q[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-    }
-};
-
-// Two 4-bit OCP E2M1 codes at once (sign bit, 2 exponent bits with bias 1,
-// 1 mantissa bit): round to nearest even with saturation at +-6, the hardware
-// conversion (its first operand goes to the high nibble); and their exact
-// values back.
-__device__ __forceinline__ uint32_t e2m1x2_codes(float lo, float hi) {
-    uint16_t r;
-    asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u16.u8 %0, t;\n}" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-__device__ __forceinline__ float2 e2m1x2_values(uint32_t codes) {
-    uint32_t h2;
-    asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}" : "=r"(h2) : "r"(codes));
-    const __half2 h = *reinterpret_cast<const __half2*>(&h2);
-    return __half22float2(h);  // .x from the low nibble
-}
 
 // kOut: write the fake-quantised W; kPack: write the packed NVFP4 nibbles (two
 // per byte, even column in the low nibble) and the block scale bytes.
@@ -108,39 +44,9 @@ __global__ void __launch_bounds__(256, 4) fake_quant_kernel(const Tin* __restric
         const float s = __fmul_rn(e4m3_value(code), g);
         float w[16];
         Vec16<Tin>::load(W + src, w);
-        // fp32(w / s): from one correctly rounded reciprocal y = RN(1/s), q = RN(w y),
-        // r = w - s q (exact, one FMA), RN(q + r y) is the correctly rounded quotient
-        // (P. Markstein, IBM J. Res. Dev. 34(1), 1990) while s is normal and no
-        // non-zero |w| is below 2^-100; other blocks divide.
-        float mn = __int_as_float(0x7F800000);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mn = (w[i] != 0.0f) ? fminf(mn, fabsf(w[i])) : mn;
-        const bool fast = s >= 1.17549435e-38f && mn >= 7.888609e-31f;
-        const float y = fast ? __frcp_rn(s) : 0.0f;
         float o[16];
-        uint32_t word[2] = {0u, 0u};
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            float u[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float wi = w[2 * p + h];
-                if (fast) {
-                    const float q0 = __fmul_rn(wi, y);
-                    // the last FMA turns -0 (w = -0) into +0; the quotient's sign is that of w
-                    u[h] = copysignf(__fmaf_rn(__fmaf_rn(-q0, s, wi), y, q0), wi);
-                } else {
-                    u[h] = (s != 0.0f) ? __fdiv_rn(wi, s) : copysignf(0.0f, wi);
-                }
-            }
-            const uint32_t c2 = e2m1x2_codes(u[0], u[1]);  // element 2p in the low nibble
-            if constexpr (kOut) {
-                const float2 q = e2m1x2_values(c2);
-                o[2 * p] = __fmul_rn(q.x, s);
-                o[2 * p + 1] = __fmul_rn(q.y, s);
-            }
-            if constexpr (kPack) word[p >> 2] |= c2 << (8 * (p & 3));
-        }
+        uint32_t word[2];
+        quantize_block<kOut, kPack>(w, s, o, word);
         if constexpr (kOut) Vec16<Tout>::store(out + 16 * b, o);
         if constexpr (kPack) {
             *reinterpret_cast<uint2*>(packed + 8 * b) = make_uint2(word[0], word[1]);
