@@ -7,11 +7,12 @@
 // tokens; the kernel contract lays H out as [cin/16, 16, 16].
 //
 // Design (B200):
-//  * Work item = (token chunk, 128-channel slab). A persistent grid walks the
-//    items; each CTA has a TMA producer warp, an MMA warp and four epilogue
-//    warps.
+//  * Work item = (token chunk, 128-channel slab). A persistent grid of two CTAs
+//    per SM walks the items; each CTA has a TMA producer warp, an MMA warp and
+//    four epilogue warps, and two CTAs per SM keep more loads in flight and fill
+//    each other's pipeline gaps.
 //  * The producer stages [128 tokens x 128 channels] bf16 tiles (two 64-channel
-//    TMA boxes, 128-byte swizzle) in a 4-deep shared-memory ring.
+//    TMA boxes, 128-byte swizzle) in a 3-deep shared-memory ring (96 KB).
 //  * The tile is channel-contiguous, so it is an MN-major operand for both
 //    A = tile^T (M = channels, K = tokens) and B = tile (K = tokens,
 //    N = channels): one tcgen05.mma (M = N = 128, K = 16, FP32 accumulate in
@@ -42,7 +43,7 @@ namespace {
 
 constexpr int kSlab = 128;                       // channels per item = MMA M = N
 constexpr int kStageTok = 128;                   // tokens per pipeline stage
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kHalfBytes = kStageTok * 64 * 2;   // one 64-channel TMA box: 16 KB
 constexpr int kStageBytes = 2 * kHalfBytes;      // 32 KB
 constexpr int kThreads = 192;                    // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
@@ -163,7 +164,7 @@ __device__ __forceinline__ bool item_chunk(const KParams& p, int64_t item, int64
     return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                  const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled tiles
@@ -584,7 +585,7 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
         attr_err = cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
     });
     if (attr_err != cudaSuccess) return cuda_status(attr_err, "set shared memory size");
-    int64_t grid = kp.n_items_max < sms ? kp.n_items_max : sms;
+    int64_t grid = kp.n_items_max < 2 * sms ? kp.n_items_max : 2 * sms;  // two CTAs per SM
     {
         // programmatic launch: the set-up of its blocks overlaps the end of the kernel before
         cudaLaunchConfig_t cfg = {};
