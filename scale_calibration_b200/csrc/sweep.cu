@@ -147,6 +147,7 @@ struct SweepShared {
     int pd[16];             // results of the shifted positive-definiteness tests
     uint32_t allow[4][kThreads];  // amax search: the codes each thread's current block may take
     float mu;               // mu <= lambda_min(D^-1/2 H D^-1/2), D = diag(H); 0 disables pruning
+    float nu;               // nu >= lambda_max(|D^-1/2 H D^-1/2|) (largest absolute row sum)
     int next_chunk;         // next 32-row chunk of the sorted order to hand to a warp
 };
 
@@ -282,6 +283,16 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             const float db = __shfl_sync(0xFFFFFFFFu, di, b, 16);
             crow[b] = (hii > 0.0f && hbb > 0.0f) ? (0.5f * (sm.Hf[i * 16 + b] + sm.Hf[b * 16 + i])) * (di * db)
                                                  : ((i == b) ? 1.0f : 0.0f);
+        }
+        // |C| is non-negative and symmetric, so its largest eigenvalue is at most its largest row
+        // sum; the entries carry a few ulps of rounding (rsqrt, products), covered by 2^-16
+        {
+            float rs = 0.0f;
+#pragma unroll
+            for (int b = 0; b < 16; ++b) rs += fabsf(crow[b]);
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) rs = fmaxf(rs, __shfl_xor_sync(0xFFFFFFFFu, rs, off));
+            if (tid == 0) sm.nu = rs * (1.0f + 1.5258789e-5f);
         }
         const float mu1 = 0.04f + 0.12f * (float)slot;
         const bool ok1 = psd_rows && shifted_pd(crow, mu1, i);
@@ -425,13 +436,14 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         if (g == 0.0f) flag = false;  // every s_c is 0: q = 0, all errors equal, code 1
 
         if (fast) {
-            // With mu > 0, H is positive semidefinite, so |H_ab| <= sqrt(H_aa H_bb) and
-            // T <= (sum_a sqrt(H_aa) |dw_a|)^2 <= 16 sum_a H_aa dw_a^2 <= 16 E / mu: the FP32
-            // error becomes relative, |E32 - E| <= rho E with rho = 16 * 48 u / mu, far tighter
+            // With mu > 0 the FP32 error of the form becomes relative. With z_a = sqrt(H_aa) dw_a
+            // and C = D^-1/2 H_s D^-1/2, T = sum |U_ab| |dw_a| |dw_b| = |z|^T |C| |z| <= nu |z|^2
+            // and E = z^T C z >= mu |z|^2, so T <= (nu / mu) E and |E32 - E| <= rho E with
+            // rho = 48 u nu / mu (nu <= 16; near 1 for weakly correlated channels), far tighter
             // than the Tw bound below for the candidates near the optimum. Thresholds then
             // follow from E in [E32 / (1 + rho), E32 / (1 - rho)]; closed forms are within 2u.
             const bool rel = sm.mu > 0.0f;
-            const float rho = rel ? fminf(768.0f * 5.9604645e-8f / sm.mu * 1.001f, 0.25f) : 0.0f;
+            const float rho = rel ? fminf(48.0f * 5.9604645e-8f * sm.nu / sm.mu * 1.001f, 0.25f) : 0.0f;
             const float up_fac = 1.0f / (1.0f - rho) * (1.0f + 4.0f * 5.9604645e-8f);  // E* <= E32 * up_fac
             // mu rounded down, less 32 u for the rounding of dw and of the bound's sum
             const float mu_lb = sm.mu * (1.0f - 32.0f * 5.9604645e-8f);
