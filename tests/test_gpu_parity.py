@@ -361,3 +361,35 @@ def test_indefinite_hessian_gets_exact_argmin(cuda_ok):
     ex, tol, fail, worst = gu.check_codes(layer.W_f32(), amax.cpu().numpy(), Hn.astype(np.float64),
                                           codes.cpu().numpy(), bam.cpu().numpy())
     assert fail == 0, (ex, tol, fail, worst)
+
+
+@pytest.mark.parametrize("kind", ["dominant_channel", "correlated", "near_collinear_pairs"])
+def test_sweep_error_bound_on_conditioned_hessians(cuda_ok, kind):
+    # Hessians whose normalised form C = D^-1/2 H D^-1/2 spans the range the FP32
+    # error bound depends on: one channel ~5000x the others (diagonal ratio ~1e7,
+    # many near ties), channels sharing a common factor (|C| row sums near 16), and
+    # pairs of almost equal channels (lambda_min(C) small); sweep-only parity
+    import scale_calibration_b200 as lh
+    rng = np.random.default_rng({"dominant_channel": 21, "correlated": 22, "near_collinear_pairs": 23}[kind])
+    c_out, c_in, n_tok = 1024, 64, 4096
+    X = rng.standard_normal((n_tok, c_in))
+    if kind == "dominant_channel":
+        X[:, rng.choice(c_in, size=4, replace=False)] *= 5000.0
+    elif kind == "correlated":
+        X = 0.3 * X + rng.standard_normal((n_tok, 1))
+    else:
+        X[:, 1::2] = X[:, 0::2] + 1e-3 * rng.standard_normal((n_tok, c_in // 2))
+    Hn = np.einsum("tja,tjb->jab", X.reshape(n_tok, c_in // 16, 16), X.reshape(n_tok, c_in // 16, 16))
+    Hn = Hn.astype(np.float32)[None]
+    Wn = (rng.standard_t(4.0, size=(c_out, c_in)) * 0.015).astype(np.float32)
+    W = torch.from_numpy(Wn).cuda()
+    H = torch.from_numpy(Hn).cuda()
+    amax = torch.empty(1, device="cuda")
+    lh.lh_absmax(W, W, 1, c_out, c_in, c_in, amax)
+    codes = torch.empty(1, c_out, c_in // 16, dtype=torch.uint8, device="cuda")
+    bam = torch.empty(1, c_out, c_in // 16, device="cuda")
+    lh.lh_sweep_scales(W, W, 1, c_out, c_in, c_in, amax, H, bam, codes)
+    torch.cuda.synchronize()
+    ex, tol, fail, worst = gu.check_codes(Wn[None], amax.cpu().numpy(), Hn.astype(np.float64),
+                                          codes.cpu().numpy(), bam.cpu().numpy())
+    assert fail == 0, (ex, tol, fail, worst)
