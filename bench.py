@@ -2,7 +2,7 @@
 """Benchmark of the Local-Hessian NVFP4 calibration hot path on B200.
 
 One step = the whole hot path for one layer, every kernel from liblh.so:
-    lh_absmax -> lh_accumulate_hessian -> lh_sweep_scales (126 candidates) -> lh_fake_quant
+    lh_absmax -> lh_accumulate_hessian -> lh_sweep_scales_ws (126 candidates) -> lh_fake_quant
 over the seeded synthetic layer (default: the attention projection,
 W [4096,4096] bf16, X [2048,4096] bf16; --config picks another).
 
@@ -234,6 +234,8 @@ def run_ours(args):
     H = torch.zeros(n_groups, J, 16, 16, dtype=torch.float32, device=dev)
     wsb = lh.lh_hessian_workspace_bytes(n_tok, c_in, n_groups)
     wsp = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    swsb = lh.lh_sweep_workspace_bytes(n_mats, c_in)
+    swsp = torch.empty(max(swsb, 16), dtype=torch.uint8, device=dev)
     codes = torch.empty(n_mats, c_out, J, dtype=torch.uint8, device=dev)
     bamax = torch.empty(n_mats, c_out, J, dtype=torch.float32, device=dev)
     Wq = torch.empty(n_mats, c_out, c_in, dtype=W.dtype, device=dev)
@@ -242,7 +244,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     s = stream.cuda_stream
     ld = W.stride(1)
-    launches_per_step = 1 + 2 + (1 if grouped else 0) + 1 + 1
+    launches_per_step = 1 + 2 + (1 if grouped else 0) + 2 + 1  # sweep: bounds kernel + sweep kernel
 
     def step(ev=None):
         H.zero_()
@@ -251,7 +253,7 @@ def run_ours(args):
         if ev: ev[1].record(stream)
         lh.lh_accumulate_hessian(X, lh.LH_BF16, n_tok, c_in, X.stride(0), off, n_groups, H, wsp, wsb, s)
         if ev: ev[2].record(stream)
-        lh.lh_sweep_scales(W, W, n_mats, c_out, c_in, ld, amax, H, bamax, codes, s)
+        lh.lh_sweep_scales_ws(W, W, n_mats, c_out, c_in, ld, amax, H, bamax, codes, swsp, swsb, s)
         if ev: ev[3].record(stream)
         lh.lh_fake_quant(W, W, n_mats, c_out, c_in, ld, amax, codes, Wq, Wq, s)
         if ev: ev[4].record(stream)
@@ -347,6 +349,7 @@ def run_ours(args):
     for _ in range(2):
         d = dict(W=torch.empty_like(W), X=torch.empty_like(X), off=torch.empty_like(off) if grouped else None,
                  amax=torch.empty_like(amax), H=torch.empty_like(H), ws=torch.empty_like(wsp),
+                 sws=torch.empty_like(swsp),
                  codes=torch.empty_like(codes), bamax=torch.empty_like(bamax), Wq=torch.empty_like(Wq),
                  codes_pin=torch.empty(codes.shape, dtype=codes.dtype).pin_memory(),
                  bam_pin=torch.empty(bamax.shape, dtype=bamax.dtype).pin_memory(),
@@ -374,7 +377,8 @@ def run_ours(args):
         lh.lh_absmax(d["W"], d["W"], n_mats, c_out, c_in, ld, d["amax"], cs)
         lh.lh_accumulate_hessian(d["X"], lh.LH_BF16, n_tok, c_in, d["X"].stride(0), d["off"], n_groups, d["H"],
                                  d["ws"], wsb, cs)
-        lh.lh_sweep_scales(d["W"], d["W"], n_mats, c_out, c_in, ld, d["amax"], d["H"], d["bamax"], d["codes"], cs)
+        lh.lh_sweep_scales_ws(d["W"], d["W"], n_mats, c_out, c_in, ld, d["amax"], d["H"], d["bamax"], d["codes"],
+                              d["sws"], swsb, cs)
         lh.lh_fake_quant(d["W"], d["W"], n_mats, c_out, c_in, ld, d["amax"], d["codes"], d["Wq"], d["Wq"], cs)
         d["ev_done"].record(s_cmp)
         with torch.cuda.stream(s_out):
@@ -499,6 +503,8 @@ def run_sharded(args):
     H = torch.zeros(n_groups, J, 16, 16, dtype=torch.float32, device=dev)
     wsb = lh.lh_hessian_workspace_bytes(max(n_loc, 1), c_in, n_groups)
     wsp = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    swsb = lh.lh_sweep_workspace_bytes(n_mats, c_in)
+    swsp = torch.empty(max(swsb, 16), dtype=torch.uint8, device=dev)
     codes = torch.empty(n_mats, rows, J, dtype=torch.uint8, device=dev)
     bamax = torch.empty(n_mats, rows, J, dtype=torch.float32, device=dev)
     Wq = torch.empty(n_mats, rows, c_in, dtype=W.dtype, device=dev)
@@ -517,7 +523,7 @@ def run_sharded(args):
             lhd.accumulate_hessian_sharded(X, n_loc, c_in, off, n_groups, H, wsp, wsb, s, check_status=False)
         else:
             lhd.allreduce_hessian(H)
-        lh.lh_sweep_scales(W, W, n_mats, rows, c_in, ld, amax, H, bamax, codes, s)
+        lh.lh_sweep_scales_ws(W, W, n_mats, rows, c_in, ld, amax, H, bamax, codes, swsp, swsb, s)
         lh.lh_fake_quant(W, W, n_mats, rows, c_in, ld, amax, codes, Wq, Wq, s)
 
     for _ in range(args.warmup):

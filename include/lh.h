@@ -170,6 +170,24 @@ LH_API lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats
                           uint8_t* best_code, void* stream);
 
 /* ------------------------------------------------------------------------
+ * lh_sweep_scales with a caller-provided workspace; the same arguments, the
+ * same results bit for bit. The workspace holds one 16-byte record per block
+ * column and matrix (the pruning bounds of its H, computed once by a first
+ * kernel instead of by every CTA of the column), and lets the launch cut its
+ * last wave of tiles into quarters; both make the call faster.
+ * workspace: device, 16-byte aligned, at least
+ *   lh_sweep_workspace_bytes(n_mats, c_in) = 16 * n_mats * (c_in / 16) bytes;
+ *   its contents on entry do not matter and are overwritten; it must not be
+ *   used by another call until this one has finished on `stream`.
+ * Errors as lh_sweep_scales, plus LH_ERR_WORKSPACE (NULL or too small) and
+ * LH_ERR_ALIGNMENT (workspace not 16-byte aligned).
+ * ---------------------------------------------------------------------- */
+LH_API size_t lh_sweep_workspace_bytes(int64_t n_mats, int64_t c_in);
+LH_API lh_status lh_sweep_scales_ws(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
+                                    int64_t ld_w, const float* global_amax, const float* H, float* best_amax,
+                                    uint8_t* best_code, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Fake quantisation with the chosen codes. "算法原理": Q(W, s) = Cast(W/s)*s.
  *   W_out[m][r][c] = cast_out( fp32( E2M1_RNE_sat(fp32(w/s)) * s ) ),
  *   s = fp32(e4m3(codes[m][r][c/16]) * fp32(global_amax[m]/2688)).

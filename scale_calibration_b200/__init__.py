@@ -4,7 +4,7 @@ The work happens in liblh.so (C ABI in include/lh.h); this package is its
 ctypes binding plus `calibrate`, which chains the four calls of the hot path
 for one layer:
 
-    lh_absmax -> lh_accumulate_hessian -> lh_sweep_scales -> lh_fake_quant
+    lh_absmax -> lh_accumulate_hessian -> lh_sweep_scales_ws -> lh_fake_quant
 
 Method: "NVIDIA Model Optimizer Local-Hessian: 基于局部 Hessian 的 NVFP4 逐块
 权重缩放算法实战指南" (xxmr.cn/news/266017), sections "算法原理" and
@@ -16,7 +16,7 @@ from ._binding import (  # noqa: F401
     EXPORTS, LH_BF16, LH_F32, LH_OK, LHError, lh_absmax, lh_accumulate_hessian, lh_fake_quant,
     lh_accumulate_hessian_noalloc, lh_debug_wait_timeout, lh_hessian_workspace_bytes, lh_last_error_message, lh_status_string,
     lh_quantize_nvfp4, lh_sweep_scales, lh_workspace_status, lh_baseline_scales, LH_SCALE_MAX,
-    LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE, lh_search_amax,
+    LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE, lh_search_amax, lh_sweep_scales_ws, lh_sweep_workspace_bytes,
 )
 
 
@@ -41,6 +41,8 @@ class Calibrator:
         self.H = torch.zeros(n_groups, J, 16, 16, dtype=torch.float32, device=device)
         self.ws_bytes = lh_hessian_workspace_bytes(n_tok, c_in, n_groups)
         self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
+        self.sweep_ws_bytes = lh_sweep_workspace_bytes(n_mats, c_in)
+        self.sweep_ws = torch.empty(max(self.sweep_ws_bytes, 16), dtype=torch.uint8, device=device)
         self.best_amax = torch.empty(n_mats, c_out, J, dtype=torch.float32, device=device)
         self.best_code = torch.empty(n_mats, c_out, J, dtype=torch.uint8, device=device)
         self.Wq = None
@@ -55,8 +57,8 @@ class Calibrator:
         lh_absmax(W, W, n_mats, c_out, c_in, W.stride(-2), self.amax, stream)
         lh_accumulate_hessian(X, LH_BF16, X.shape[0], c_in, X.stride(0), offsets if self.grouped else None,
                               self.n_groups, self.H, self.ws, self.ws_bytes, stream)
-        lh_sweep_scales(W, W, n_mats, c_out, c_in, W.stride(-2), self.amax, self.H, self.best_amax,
-                        self.best_code, stream)
+        lh_sweep_scales_ws(W, W, n_mats, c_out, c_in, W.stride(-2), self.amax, self.H, self.best_amax,
+                           self.best_code, self.sweep_ws, self.sweep_ws_bytes, stream)
         lh_fake_quant(W, W, n_mats, c_out, c_in, W.stride(-2), self.amax, self.best_code, self.Wq, self.Wq, stream)
         return self.best_code, self.best_amax, self.Wq
 

@@ -20,7 +20,7 @@ EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
     "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout", "lh_quantize_nvfp4", "lh_baseline_scales",
-    "lh_search_amax",
+    "lh_search_amax", "lh_sweep_workspace_bytes", "lh_sweep_scales_ws",
 ]
 LH_SCALE_MAX, LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE = range(3)
 
@@ -46,6 +46,8 @@ def _load() -> ctypes.CDLL:
         "lh_accumulate_hessian_noalloc": (I32, [P, I32, I64, I64, I64, P, I64, P, P]),
         "lh_debug_wait_timeout": (I32, [P, ctypes.c_size_t, I64, I32, P]),
         "lh_sweep_scales": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P]),
+        "lh_sweep_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
+        "lh_sweep_scales_ws": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P, ctypes.c_size_t, P]),
         "lh_fake_quant": (I32, [P, I32, I64, I64, I64, I64, P, P, P, I32, P]),
         "lh_quantize_nvfp4": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P, P, I32, P]),
         "lh_baseline_scales": (I32, [P, I32, I64, I64, I64, I64, P, I32, P, P, P]),
@@ -154,6 +156,19 @@ def lh_sweep_scales(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, H, best_
                              _ptr(best_amax), _ptr(best_code), _stream(stream))
     if check:
         _check(s, "lh_sweep_scales")
+    return s
+
+
+def lh_sweep_workspace_bytes(n_mats, c_in) -> int:
+    return int(_lib.lh_sweep_workspace_bytes(n_mats, c_in))
+
+
+def lh_sweep_scales_ws(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, H, best_amax, best_code, workspace,
+                       workspace_bytes, stream=None, check=True) -> int:
+    s = _lib.lh_sweep_scales_ws(_ptr(W), _dtype(w_dtype), n_mats, c_out, c_in, ld_w, _ptr(global_amax), _ptr(H),
+                                _ptr(best_amax), _ptr(best_code), _ptr(workspace), workspace_bytes, _stream(stream))
+    if check:
+        _check(s, "lh_sweep_scales_ws")
     return s
 
 

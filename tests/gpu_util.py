@@ -23,7 +23,7 @@ def to_device(layer: synth.Layer):
 
 
 def run_library(layer: synth.Layer, out_dtype=None, W=None, X=None, off=None):
-    """absmax -> Hessian -> sweep -> fake-quant through the C ABI; numpy results."""
+    """absmax -> Hessian -> sweep (with its workspace) -> fake-quant through the C ABI; numpy results."""
     import scale_calibration_b200 as lh
     if W is None:
         W, X, off = to_device(layer)
@@ -39,7 +39,14 @@ def run_library(layer: synth.Layer, out_dtype=None, W=None, X=None, off=None):
     assert lh.lh_workspace_status(ws) == 0
     codes = torch.empty(n_mats, c_out, J, dtype=torch.uint8, device="cuda")
     bamax = torch.empty(n_mats, c_out, J, dtype=torch.float32, device="cuda")
-    lh.lh_sweep_scales(W, W, n_mats, c_out, c_in, W.stride(1), amax, H, bamax, codes)
+    # the product path takes the sweep's workspace; the call without one must agree bit for bit
+    swsb = lh.lh_sweep_workspace_bytes(n_mats, c_in)
+    sws = torch.empty(max(swsb, 16), dtype=torch.uint8, device="cuda")
+    lh.lh_sweep_scales_ws(W, W, n_mats, c_out, c_in, W.stride(1), amax, H, bamax, codes, sws, swsb)
+    codes2 = torch.empty_like(codes)
+    bamax2 = torch.empty_like(bamax)
+    lh.lh_sweep_scales(W, W, n_mats, c_out, c_in, W.stride(1), amax, H, bamax2, codes2)
+    assert torch.equal(codes, codes2) and torch.equal(bamax.view(torch.int32), bamax2.view(torch.int32))
     od = out_dtype or W.dtype
     Wq = torch.empty(n_mats, c_out, c_in, dtype=od, device="cuda")
     lh.lh_fake_quant(W, W, n_mats, c_out, c_in, W.stride(1), amax, codes, Wq, Wq)

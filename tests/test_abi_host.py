@@ -54,6 +54,25 @@ def test_sweep_rejects_bad_arguments():
         assert lh.lh_last_error_message() != ""
 
 
+def test_sweep_ws_rejects_bad_arguments():
+    lh = _lh()
+    need = lh.lh_sweep_workspace_bytes(2, 128)
+    assert need == 16 * 2 * 8
+    assert lh.lh_sweep_workspace_bytes(0, 128) == 0 and lh.lh_sweep_workspace_bytes(1, 24) == 0
+    ok = dict(W=FAKE, w_dtype=lh.LH_BF16, n_mats=2, c_out=64, c_in=128, ld_w=128, global_amax=FAKE, H=FAKE,
+              best_amax=FAKE, best_code=FAKE, workspace=FAKE, workspace_bytes=need, stream=0, check=False)
+    cases = [
+        (dict(workspace=0), 4), (dict(workspace_bytes=need - 1), 4), (dict(workspace=FAKE + 8), 3),
+        (dict(W=0), 1), (dict(n_mats=0), 1), (dict(c_in=24, ld_w=24), 2), (dict(W=FAKE + 2), 3), (dict(w_dtype=7), 2),
+    ]
+    for over, want in cases:
+        a = dict(ok, **over)
+        assert lh.lh_sweep_scales_ws(**a) == want, over
+        assert lh.lh_last_error_message() != ""
+    # nothing to sweep: no launch, whatever the sizes
+    assert lh.lh_sweep_scales_ws(**dict(ok, c_out=0)) == 0
+
+
 def test_sweep_empty_is_noop():
     lh = _lh()
     assert lh.lh_sweep_scales(FAKE, lh.LH_BF16, 1, 0, 128, 128, FAKE, FAKE, FAKE, FAKE, 0, check=False) == 0

@@ -393,3 +393,42 @@ def test_sweep_error_bound_on_conditioned_hessians(cuda_ok, kind):
     ex, tol, fail, worst = gu.check_codes(Wn[None], amax.cpu().numpy(), Hn.astype(np.float64),
                                           codes.cpu().numpy(), bam.cpu().numpy())
     assert fail == 0, (ex, tol, fail, worst)
+
+
+@pytest.mark.parametrize("c_out,c_in,n_mats,h_none", [(1, 16, 1, False), (700, 48, 3, False), (2100, 32, 1, True),
+                                                     (4096, 2560, 1, False)])
+def test_sweep_workspace_variant_matches(cuda_ok, c_out, c_in, n_mats, h_none):
+    # the workspace path (column bounds from a first kernel) returns what the path
+    # without a workspace returns, on shapes where every tile or only the last wave
+    # of tiles is halved, ragged tiles, several matrices and the identity H; stale
+    # workspace contents do not matter
+    import scale_calibration_b200 as lh
+    rng = np.random.default_rng(c_out + c_in)
+    Wn = (rng.standard_t(4.0, size=(n_mats, c_out, c_in)) * 0.015).astype(np.float32)
+    W = torch.from_numpy(Wn).cuda().to(torch.bfloat16)
+    X = rng.standard_normal((512, c_in)) * rng.lognormal(0.0, 1.0, size=c_in)
+    Hn = np.einsum("tja,tjb->jab", X.reshape(512, c_in // 16, 16), X.reshape(512, c_in // 16, 16)).astype(np.float32)
+    H = None if h_none else torch.from_numpy(np.broadcast_to(Hn, (n_mats,) + Hn.shape).copy()).cuda()
+    amax = torch.empty(n_mats, device="cuda")
+    lh.lh_absmax(W, W, n_mats, c_out, c_in, c_in, amax)
+    J = c_in // 16
+    out = []
+    for use_ws in (False, True):
+        codes = torch.empty(n_mats, c_out, J, dtype=torch.uint8, device="cuda")
+        bam = torch.empty(n_mats, c_out, J, device="cuda")
+        if use_ws:
+            wsb = lh.lh_sweep_workspace_bytes(n_mats, c_in)
+            ws = torch.full((wsb,), 0x7F, dtype=torch.uint8, device="cuda")
+            lh.lh_sweep_scales_ws(W, W, n_mats, c_out, c_in, c_in, amax, H, bam, codes, ws, wsb)
+        else:
+            lh.lh_sweep_scales(W, W, n_mats, c_out, c_in, c_in, amax, H, bam, codes)
+        torch.cuda.synchronize()
+        out.append((codes.cpu().numpy(), bam.cpu().numpy()))
+    assert np.array_equal(out[0][0], out[1][0])
+    assert np.array_equal(out[0][1].view(np.int32), out[1][1].view(np.int32))
+    if c_out * J * n_mats <= 20000:
+        Hd = (np.broadcast_to(np.eye(16), (n_mats, J, 16, 16)) if h_none
+              else np.broadcast_to(Hn, (n_mats,) + Hn.shape)).astype(np.float64)
+        Wf = W.float().cpu().numpy()
+        ex, tol, fail, worst = gu.check_codes(Wf, amax.cpu().numpy(), Hd, out[1][0], out[1][1])
+        assert fail == 0, (ex, tol, fail, worst)
