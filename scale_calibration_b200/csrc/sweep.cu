@@ -9,19 +9,28 @@
 // amax out.
 //
 // Design (B200, FP32 CUDA cores):
-//  * One thread owns one block (row r, block column j); a CTA covers 128 rows
-//    of one block column, so the 16x16 H_j is staged once in shared memory
-//    and read by broadcast.
-//  * Candidate scales come in 8 mantissa classes m * 2^x (m = 1 + f/8). Within
-//    a class, consecutive codes double the scale exactly, so fp32(w / s_c) is
-//    fp32(w / s_c0) scaled by a power of two: 16 IEEE divisions per class
-//    replace 16 per candidate, and each candidate rounds the same quotient
-//    onto the E2M1 grid scaled by 2^k (exact, see e2m1_grid_round).
-//  * E(c) is evaluated in FP32 with the symmetric form (136 FMA). Its
-//    rounding error is at most ~35 u * sum|dw_a||H_ab||dw_b| (u = 2^-24), and
-//    |dw_i| <= |w_i|, so every block whose runner-up is within twice that bound
-//    of the best is re-swept in FP64 by the whole warp. The result is the
-//    exact argmin (up to FP64 rounding), lowest code on ties.
+//  * One thread owns one block (row r, block column j). A CTA of 128 threads
+//    takes a tile of 1024 rows of one block column (the last wave of tiles is
+//    cut into 512-row halves so the launch drains quickly), stages H_j once in
+//    shared memory (read by broadcast), sorts the tile's rows by the largest
+//    |w| over the heavy channels, and hands out 32-row chunks of the sorted
+//    order to its four warps.
+//  * Candidate scales come in 8 mantissa classes (1 + f/8) * 2^x. Within a
+//    class consecutive codes double the scale exactly, so fp32(w / s_c) is
+//    fp32(w / s_c0) scaled by a power of two: 16 correctly rounded quotients
+//    per class replace 16 per candidate, and each candidate rounds them onto
+//    the E2M1 grid scaled by 2^k (exact).
+//  * Per class a warp walks up and down from its max-scaling step. A lower
+//    bound mu * sum_a H_aa dw_a^2 <= E skips the form for candidates that
+//    cannot win, and class-wide bounds end each direction early; mu comes from
+//    shifted Cholesky tests of the normalised H (per CTA, or once per column by
+//    a first kernel when the caller gives a workspace).
+//  * The survivors' E(c) is evaluated in FP32 with the symmetric form (136
+//    FMA). Its error is at most rho * E with rho = 48 u nu / mu (nu bounds the
+//    largest eigenvalue of |normalised H|), or an absolute bound when mu = 0;
+//    blocks whose runner-up is within that bound of the best are re-swept in
+//    FP64 by the whole warp. The result is the exact argmin (up to FP64
+//    rounding), lowest code on ties.
 #include <cmath>
 
 #include "common.cuh"
