@@ -11,7 +11,7 @@
 // Design (B200, FP32 CUDA cores):
 //  * One thread owns one block (row r, block column j). A CTA of 128 threads
 //    takes a tile of 1024 rows of one block column (the last wave of tiles is
-//    cut into 512-row halves so the launch drains quickly), stages H_j once in
+//    cut into 512- and 256-row pieces so the launch drains quickly), stages H_j once in
 //    shared memory (read by broadcast), sorts the tile's rows by the largest
 //    |w| over the heavy channels, and hands out 32-row chunks of the sorted
 //    order to its four warps.
@@ -142,38 +142,46 @@ static_assert(kPairSlots == 72, "72 padded pair slots");
 constexpr int kTileRows = kThreads * kRowsPerThread;  // rows of one CTA, walked in sorted order
 
 constexpr int kSortBuckets = 512;
-constexpr int kParts = 2;
-constexpr int kQuarter = kTileRows / kParts;  // rows of a split tile (512)
 
 // Work units of one launch, in launch order: the tiles (kTileRows rows of one block
-// column, column-major over (m, j)), of which the last n_split are cut into halves.
-// CTAs start in launch order, so the halves run last and the final wave drains in
-// half a tile's time. Large tiles sort more rows together (the warps of a tile agree
-// more on where their walks start and stop) and spread the per-CTA set-up over more
-// rows; halves keep the drain at the cost of a 512-row tile.
+// column, column-major over (m, j)); of the last wave of tiles, the first three
+// quarters are cut into halves and the rest into quarters. CTAs start in launch
+// order, so the pieces run last and the launch drains in a fraction of a tile's time.
+// Large tiles sort more rows together (the warps of a tile agree more on where their
+// walks start and stop) and spread the per-CTA set-up over more rows; pieces of
+// fewer rows walk more slowly per row, so only the very end is cut finest.
 struct Units {
     int64_t tiles_per_col;  // ceil(c_out / kTileRows)
     int64_t n_tiles;        // tiles_per_col * J * n_mats
-    int64_t n_split;        // tiles cut into quarters (the last ones)
+    int64_t n_split;        // tiles cut into halves
+    int64_t n_quart;        // tiles after those, cut into quarters (the last ones)
 };
 
 __device__ __forceinline__ void unit_of(const Units& U, int64_t J, int64_t c_out, int64_t u, int64_t& m, int64_t& j,
                                         int64_t& row0, int& nrows) {
-    const int64_t whole = U.n_tiles - U.n_split;
-    int64_t t, q0 = 0, qn = kParts;
+    const int64_t whole = U.n_tiles - U.n_split - U.n_quart;
+    int64_t t, r0, rn;
     if (u < whole) {
         t = u;
+        r0 = 0;
+        rn = kTileRows;
+    } else if (u < whole + 2 * U.n_split) {
+        const int64_t v = u - whole;
+        t = whole + v / 2;
+        r0 = (v % 2) * (kTileRows / 2);
+        rn = kTileRows / 2;
     } else {
-        t = whole + (u - whole) / kParts;
-        q0 = (u - whole) % kParts;
-        qn = 1;
+        const int64_t v = u - whole - 2 * U.n_split;
+        t = whole + U.n_split + v / 4;
+        r0 = (v % 4) * (kTileRows / 4);
+        rn = kTileRows / 4;
     }
     const int64_t col = t / U.tiles_per_col;
     m = col / J;
     j = col - m * J;
-    row0 = (t - col * U.tiles_per_col) * kTileRows + q0 * kQuarter;
+    row0 = (t - col * U.tiles_per_col) * kTileRows + r0;
     const int64_t left = c_out - row0;
-    nrows = left <= 0 ? 0 : (int)(left < qn * kQuarter ? left : qn * kQuarter);
+    nrows = left <= 0 ? 0 : (int)(left < rn ? left : rn);
 }
 
 // The pruning bounds of one block column (mu, nu below), computed once per column by
@@ -880,11 +888,13 @@ lh_status launch_sweep(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t 
     Units U;
     U.tiles_per_col = (c_out + kTileRows - 1) / kTileRows;
     U.n_tiles = U.tiles_per_col * J * n_mats;
-    // one wave of tiles (4 resident CTAs per SM at 128 registers) cut into halves: the
-    // whole tiles started last end while the halves still keep every SM busy
+    // one wave of tiles (4 resident CTAs per SM at 128 registers) cut into pieces: the
+    // whole tiles started last end while the pieces still keep every SM busy
     const int64_t slots = 4 * (int64_t)sm_count();
-    U.n_split = U.n_tiles < slots ? U.n_tiles : slots;
-    const int64_t n_units = U.n_tiles + (kParts - 1) * U.n_split;
+    const int64_t n_cut = U.n_tiles < slots ? U.n_tiles : slots;
+    U.n_quart = n_cut / 4;
+    U.n_split = n_cut - U.n_quart;
+    const int64_t n_units = U.n_tiles + U.n_split + 3 * U.n_quart;
     if (n_units > 0x7FFFFFFF)
         return fail(LH_ERR_UNSUPPORTED, "too many blocks: ceil(c_out/512) * c_in/16 * n_mats must be < 2^31");
     const dim3 grid((unsigned)n_units);
