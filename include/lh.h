@@ -172,9 +172,8 @@ LH_API lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats
 /* ------------------------------------------------------------------------
  * lh_sweep_scales with a caller-provided workspace; the same arguments, the
  * same results bit for bit. The workspace holds one 16-byte record per block
- * column and matrix (the pruning bounds of its H, computed once by a first
- * kernel instead of by every CTA of the column), and lets the launch cut its
- * last wave of tiles into quarters; both make the call faster.
+ * column and matrix: the pruning bounds of its H, computed once by a first
+ * kernel instead of by every CTA of the column, which makes the call faster.
  * workspace: device, 16-byte aligned, at least
  *   lh_sweep_workspace_bytes(n_mats, c_in) = 16 * n_mats * (c_in / 16) bytes;
  *   its contents on entry do not matter and are overwritten; it must not be
