@@ -282,6 +282,24 @@ def run_ours(args):
     t_all = max_over_ranks(t_rank, ws, dev)
     value = n_mats * c_out * J * ws * args.steps / t_all
     t_abs, t_hess, t_sweep, t_fq = (float(x) for x in per.mean(axis=0))  # ms
+    names = ("absmax", "hessian", "sweep", "fake_quant")
+    per_median = {n: float(v) for n, v in zip(names, np.median(per, axis=0))}
+    per_min = {n: float(v) for n, v in zip(names, per.min(axis=0))}
+
+    # ---- the Hessian call with X left in L2 (no flush between calls): X of the attention,
+    # MLP-up and MoE layers (17, 67, 134 MB) fits or nearly fits the 126 MB L2
+    warm = []
+    for i in range(3 + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        lh.lh_accumulate_hessian(X, lh.LH_BF16, n_tok, c_in, X.stride(0), off, n_groups, H, wsp, wsb, s)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= 3:
+            warm.append(e0.elapsed_time(e1))
+    t_hess_warm = float(np.median(warm))
+    H.zero_()  # back to one accumulation (deterministic: the same H as the timed steps)
+    lh.lh_accumulate_hessian(X, lh.LH_BF16, n_tok, c_in, X.stride(0), off, n_groups, H, wsp, wsb, s)
 
     # ---- packed NVFP4 export fused with the fake quantisation (one read of W writes the
     # packed nibbles, the scale bytes and W_q), timed like the step, L2 flushed each time
@@ -433,7 +451,11 @@ def run_ours(args):
                    achieved=hess_gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=hess_gbs / peaks["hbm_gbs"],
                    bytes_per_launch=hess_bytes, peak_source=peaks["source"],
                    traffic=profiled_traffic("scale_calibration_b200/csrc/hessian.cu", "hessian_tc_kernel_mlp_down.md")
-                   if args.config == 3 else None)
+                   if args.config == 3 else None,
+                   warm_l2=dict(ms=t_hess_warm, tokens_per_s=n_tok * ws / (t_hess_warm / 1e3),
+                                achieved=hess_bytes / (t_hess_warm / 1e3) / 1e9,
+                                note="median of back-to-back calls without an L2 flush (X partly or wholly in L2); "
+                                     "the HBM fraction above is the cold-L2 one"))
 
     line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=ws, steps=args.steps, warmup=args.warmup,
                 ms_per_step=1e3 * t_all / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None,
@@ -441,6 +463,7 @@ def run_ours(args):
                 config=dict(workload=workload_desc(layer), blocks=n_blocks, tokens=n_tok, l2="flushed",
                             parallelism=f"{ws} independent layers, no collective"),
                 kernels_ms=dict(absmax=t_abs, hessian=t_hess, sweep=t_sweep, fake_quant=t_fq),
+                kernels_ms_median=per_median, kernels_ms_min=per_min,
                 baseline_scalers=baselines,
                 nvfp4_export=dict(ms=t_ex, bytes_per_launch=int(ex_bytes), bound="hbm",
                                   achieved=ex_bytes / (t_ex / 1e3) / 1e9, unit="GB/s",
