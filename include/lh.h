@@ -161,8 +161,10 @@ LH_API lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, 
  * proven bound on the FP32 rounding error are re-evaluated in FP64, so the
  * chosen code is the exact argmin up to FP64 rounding.
  * W: device bf16 or f32 [n_mats][c_out][ld_w]. global_amax: device f32 [n_mats].
- * H: device f32 [n_mats][c_in/16][16][16] (symmetric; the upper triangle is read), or NULL
- *   for the identity (the weight-MSE sweep of the pages' MSE baseline).
+ * H: device f32 [n_mats][c_in/16][16][16] (both triangles are read; E depends on the
+ *   symmetric part (H + H^T)/2 only, so a symmetric H from lh_accumulate_hessian and any
+ *   matrix with the same symmetric part give the same codes), or NULL for the identity
+ *   (the weight-MSE sweep of the pages' MSE baseline).
  * best_amax: device f32 [n_mats][c_out][c_in/16]. best_code: device u8, same shape.
  * ---------------------------------------------------------------------- */
 LH_API lh_status lh_sweep_scales(const void* W, lh_dtype w_dtype, int64_t n_mats, int64_t c_out, int64_t c_in,
