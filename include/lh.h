@@ -160,7 +160,9 @@ LH_API lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, 
  * E is evaluated in FP32; blocks whose two best candidates are closer than a
  * proven bound on the FP32 rounding error are re-evaluated in FP64, so the
  * chosen code is the exact argmin up to FP64 rounding.
- * W: device bf16 or f32 [n_mats][c_out][ld_w]. global_amax: device f32 [n_mats].
+ * W: device bf16 or f32 [n_mats][c_out][ld_w]. global_amax: device f32 [n_mats], finite
+ *   and >= 0 (as lh_absmax writes it); 0 is defined (every block gets code 1 and amax 0);
+ *   a NaN, infinite or negative value is not detected and gives unspecified codes.
  * H: device f32 [n_mats][c_in/16][16][16] (both triangles are read; E depends on the
  *   symmetric part (H + H^T)/2 only, so a symmetric H from lh_accumulate_hessian and any
  *   matrix with the same symmetric part give the same codes), or NULL for the identity
