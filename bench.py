@@ -591,7 +591,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=1, help="0 tiny, 1 attn_proj, 2 mlp_up, 3 mlp_down, 4 moe_experts")
+    ap.add_argument("--config", type=int, default=4, help="0 tiny, 1 attn_proj, 2 mlp_up, 3 mlp_down, 4 moe_experts (default: the largest single-GPU layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--mode", choices=["layers", "sharded"], default="layers",
