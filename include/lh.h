@@ -135,13 +135,25 @@ LH_API lh_status lh_debug_wait_timeout(void* workspace, size_t workspace_bytes, 
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
+ *   - Argument errors are the same, checked in the same order, as those of
+ *     lh_accumulate_hessian; the size limit is checked after them.
  *   - All calls share the array (it keeps the last call's contents; what must
  *     start at zero is cleared by each call). Calls whose kernels overlap on
  *     the GPU race on it: serialise them (one stream, one thread at a time).
+ *   - Errors the kernels find (an expired bounded wait, overlapping group
+ *     offsets) are written to the array's header, not returned: read them with
+ *     lh_noalloc_status after the call, before the next allocation-free call on
+ *     that device clears them.
  * ---------------------------------------------------------------------- */
 LH_API lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, int64_t n_tokens_total,
                                                int64_t c_in, int64_t ld_x, const int64_t* offsets,
                                                int64_t n_groups, float* H, void* stream);
+
+/* Status the last lh_accumulate_hessian_noalloc call on the current device left
+ * in the library's scratch array: LH_OK, LH_ERR_TIMEOUT or LH_ERR_INVALID_ARG
+ * with the meaning lh_workspace_status gives them. Synchronises `stream` (pass
+ * the stream of that call). The pages have no counterpart. */
+LH_API lh_status lh_noalloc_status(void* stream);
 
 /* ------------------------------------------------------------------------
  * FP8 block-scale sweep. "算法原理": per 16-weight block, all 126 FP8 E4M3

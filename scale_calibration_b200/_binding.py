@@ -19,7 +19,7 @@ LH_BF16, LH_F32 = 0, 1
 EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
-    "lh_accumulate_hessian_noalloc", "lh_debug_wait_timeout", "lh_quantize_nvfp4", "lh_baseline_scales",
+    "lh_accumulate_hessian_noalloc", "lh_noalloc_status", "lh_debug_wait_timeout", "lh_quantize_nvfp4", "lh_baseline_scales",
     "lh_search_amax", "lh_sweep_workspace_bytes", "lh_sweep_scales_ws",
 ]
 LH_SCALE_MAX, LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE = range(3)
@@ -44,6 +44,7 @@ def _load() -> ctypes.CDLL:
         "lh_accumulate_hessian": (I32, [P, I32, I64, I64, I64, P, I64, P, P, ctypes.c_size_t, P]),
         "lh_workspace_status": (I32, [P, P]),
         "lh_accumulate_hessian_noalloc": (I32, [P, I32, I64, I64, I64, P, I64, P, P]),
+        "lh_noalloc_status": (I32, [P]),
         "lh_debug_wait_timeout": (I32, [P, ctypes.c_size_t, I64, I32, P]),
         "lh_sweep_scales": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P]),
         "lh_sweep_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
@@ -148,6 +149,10 @@ def lh_debug_wait_timeout(workspace, workspace_bytes, timeout_us, arrive, stream
 
 def lh_workspace_status(workspace, stream=None) -> int:
     return _lib.lh_workspace_status(_ptr(workspace), _stream(stream))
+
+
+def lh_noalloc_status(stream=None) -> int:
+    return _lib.lh_noalloc_status(_stream(stream))
 
 
 def lh_sweep_scales(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, H, best_amax, best_code, stream=None,

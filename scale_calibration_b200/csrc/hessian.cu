@@ -460,6 +460,23 @@ __global__ void __launch_bounds__(256) hessian_reduce1_kernel(const float* __res
     *h = (float)((double)*h + s);
 }
 
+// Argument checks shared by the Hessian entry points (host side, before any launch).
+lh_status validate_hessian_args(const void* X, lh_dtype x_dtype, int64_t n_tokens_total, int64_t c_in, int64_t ld_x,
+                                const int64_t* offsets, int64_t n_groups, const float* H) {
+    if (x_dtype != LH_BF16) return fail(LH_ERR_UNSUPPORTED, "X must be LH_BF16");
+    if (!X || !H) return fail(LH_ERR_INVALID_ARG, "null X or H");
+    if (n_tokens_total < 0 || c_in < 0 || n_groups < 1)
+        return fail(LH_ERR_INVALID_ARG, "n_tokens_total, c_in must be >= 0 and n_groups >= 1");
+    if (!offsets && n_groups != 1) return fail(LH_ERR_INVALID_ARG, "offsets == NULL requires n_groups == 1");
+    if (c_in % 16 != 0) return fail(LH_ERR_UNSUPPORTED, "c_in=%lld is not a multiple of 16", (long long)c_in);
+    if (ld_x < c_in) return fail(LH_ERR_INVALID_ARG, "ld_x < c_in");
+    if (!aligned16(X) || (ld_x * 2) % 16 != 0)
+        return fail(LH_ERR_ALIGNMENT, "X must be 16-byte aligned and ld_x a multiple of 8");
+    if (n_tokens_total >= ((int64_t)1 << 31) || c_in >= ((int64_t)1 << 31) || n_groups > 65535)
+        return fail(LH_ERR_UNSUPPORTED, "n_tokens_total and c_in must be < 2^31, n_groups <= 65535");
+    return LH_OK;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     static std::once_flag once;
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -518,17 +535,8 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
                                            void* workspace, size_t workspace_bytes, void* stream) {
     using namespace lh;
     clear_error();
-    if (x_dtype != LH_BF16) return fail(LH_ERR_UNSUPPORTED, "X must be LH_BF16");
-    if (!X || !H) return fail(LH_ERR_INVALID_ARG, "null X or H");
-    if (n_tokens_total < 0 || c_in < 0 || n_groups < 1)
-        return fail(LH_ERR_INVALID_ARG, "n_tokens_total, c_in must be >= 0 and n_groups >= 1");
-    if (!offsets && n_groups != 1) return fail(LH_ERR_INVALID_ARG, "offsets == NULL requires n_groups == 1");
-    if (c_in % 16 != 0) return fail(LH_ERR_UNSUPPORTED, "c_in=%lld is not a multiple of 16", (long long)c_in);
-    if (ld_x < c_in) return fail(LH_ERR_INVALID_ARG, "ld_x < c_in");
-    if (!aligned16(X) || (ld_x * 2) % 16 != 0)
-        return fail(LH_ERR_ALIGNMENT, "X must be 16-byte aligned and ld_x a multiple of 8");
-    if (n_tokens_total >= ((int64_t)1 << 31) || c_in >= ((int64_t)1 << 31) || n_groups > 65535)
-        return fail(LH_ERR_UNSUPPORTED, "n_tokens_total and c_in must be < 2^31, n_groups <= 65535");
+    lh_status s = validate_hessian_args(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H);
+    if (s != LH_OK) return s;
     if (n_tokens_total == 0 || c_in == 0) return LH_OK;
     const Plan plan = make_plan(n_tokens_total, c_in, n_groups);
     if (!workspace || workspace_bytes < plan.ws.total)
@@ -553,7 +561,7 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    lh_status s = cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, st), "clear workspace header");
+    s = cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, st), "clear workspace header");
     if (s != LH_OK) return s;
 
     const int64_t J = c_in / 16;
@@ -656,35 +664,54 @@ void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
 
 static __device__ __align__(256) unsigned char lh_noalloc_scratch[kNoAllocScratchBytes];
 
+// Device address of the scratch array for the current device, looked up on
+// first use with that device current (the only set-up the entry point needs).
+static lh_status noalloc_scratch(void** out) {
+    using namespace lh;
+    int dev = 0;
+    lh_status s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
+    if (s != LH_OK) return s;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(LH_ERR_UNSUPPORTED, "device index %d too large", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        s = cuda_status(cudaGetSymbolAddress(&p, lh_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+        if (s != LH_OK) return s;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LH_OK;
+}
+
 extern "C" lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, int64_t n_tokens_total,
                                                    int64_t c_in, int64_t ld_x, const int64_t* offsets,
                                                    int64_t n_groups, float* H, void* stream) {
     using namespace lh;
     clear_error();
+    // the same argument checks, in the same order, as the workspace entry point
+    lh_status s = validate_hessian_args(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H);
+    if (s != LH_OK) return s;
+    if (n_tokens_total == 0 || c_in == 0) return LH_OK;
     const size_t need = lh_hessian_workspace_bytes(n_tokens_total, c_in, n_groups);
-    if (n_tokens_total == 0 || c_in == 0 || need == 0)  // no-op or invalid sizes: the checks of the main entry
-        return lh_accumulate_hessian(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H, nullptr, 0,
-                                     stream);
     if (need > kNoAllocScratchBytes)
         return fail(LH_ERR_WORKSPACE,
                     "this Hessian needs %zu bytes of scratch but the allocation-free entry point has %zu "
                     "(16 MiB); call lh_accumulate_hessian with a caller-provided workspace instead",
                     need, kNoAllocScratchBytes);
-    int dev = 0;
-    lh_status s = cuda_status(cudaGetDevice(&dev), "cudaGetDevice");
-    if (s != LH_OK) return s;
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(LH_ERR_UNSUPPORTED, "device index %d too large", dev);
     void* scratch = nullptr;
-    {
-        std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {
-            void* p = nullptr;
-            s = cuda_status(cudaGetSymbolAddress(&p, lh_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
-            if (s != LH_OK) return s;
-            g_noalloc_ptr[dev] = p;
-        }
-        scratch = g_noalloc_ptr[dev];
-    }
+    s = noalloc_scratch(&scratch);
+    if (s != LH_OK) return s;
     return lh_accumulate_hessian(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H, scratch,
                                  kNoAllocScratchBytes, stream);
+}
+
+// Status the last allocation-free call on the current device left in the
+// scratch array's header; the same words lh_workspace_status reads.
+extern "C" lh_status lh_noalloc_status(void* stream) {
+    using namespace lh;
+    clear_error();
+    void* scratch = nullptr;
+    lh_status s = noalloc_scratch(&scratch);
+    if (s != LH_OK) return s;
+    return lh_workspace_status(scratch, stream);
 }

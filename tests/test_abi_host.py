@@ -94,6 +94,30 @@ def test_hessian_rejects_bad_arguments():
         assert lh.lh_accumulate_hessian(**a) == want, over
 
 
+def test_hessian_noalloc_checks_arguments_like_the_workspace_entry():
+    # the allocation-free entry point returns the same argument errors, before its size limit
+    # and before touching any device (no GPU here)
+    lh = _lh()
+    ok = dict(X=FAKE, x_dtype=lh.LH_BF16, n_tokens_total=300, c_in=64, ld_x=64, offsets=None, n_groups=1, H=FAKE,
+              stream=0, check=False)
+    cases = [
+        (dict(x_dtype=lh.LH_F32), 2), (dict(X=0), 1), (dict(H=0), 1), (dict(n_groups=2), 1),
+        (dict(c_in=40, ld_x=40), 2), (dict(ld_x=60), 1), (dict(ld_x=68), 3), (dict(X=FAKE + 8), 3),
+        (dict(n_tokens_total=-1), 1), (dict(n_groups=0), 1),
+        # far beyond the 16 MiB scratch, but the argument error comes first
+        (dict(n_tokens_total=1 << 24, c_in=40008, ld_x=40008), 2),
+        (dict(n_tokens_total=1 << 24, c_in=32768, ld_x=32768, X=0), 1),
+    ]
+    for over, want in cases:
+        a = dict(ok, **over)
+        assert lh.lh_accumulate_hessian_noalloc(**a) == want, over
+    # valid arguments beyond the scratch: LH_ERR_WORKSPACE, still before any device call
+    a = dict(ok, n_tokens_total=1 << 24, c_in=32768, ld_x=32768)
+    assert lh.lh_accumulate_hessian_noalloc(**a) == 4
+    assert "16 MiB" in lh.lh_last_error_message()
+    assert lh.lh_accumulate_hessian_noalloc(**dict(ok, n_tokens_total=0)) == 0
+
+
 def test_hessian_zero_tokens_is_noop():
     lh = _lh()
     assert lh.lh_accumulate_hessian(FAKE, lh.LH_BF16, 0, 64, 64, None, 1, FAKE, 0, 0, 0, check=False) == 0

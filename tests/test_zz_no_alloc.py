@@ -28,8 +28,10 @@ def _hessians(layer):
     wsb = lh.lh_hessian_workspace_bytes(layer.n_tok, layer.c_in, n_groups)
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
     lh.lh_accumulate_hessian(X, lh.LH_BF16, layer.n_tok, layer.c_in, X.stride(0), off, n_groups, H_ws, ws, wsb)
+    assert lh.lh_workspace_status(ws) == 0
     H_na = torch.zeros_like(H_ws)
     lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, layer.n_tok, layer.c_in, X.stride(0), off, n_groups, H_na)
+    assert lh.lh_noalloc_status() == 0  # no kernel-side error left in the scratch header
     torch.cuda.synchronize()
     return H_ws.cpu().numpy(), H_na.cpu().numpy()
 
@@ -44,6 +46,23 @@ def test_noalloc_matches_workspace_entry_on_consecutive_calls(cuda_ok):
         per, whole, bad = gu.hessian_rel_errors(H_na, H_ws.astype(np.float64))
         assert per <= gu.HESSIAN_RTOL and whole <= gu.HESSIAN_RTOL and bad == 0, (per, whole, bad)
         assert np.array_equal(H_ws, H_na)  # same kernels, deterministic order
+
+
+def test_noalloc_reports_kernel_side_errors_through_its_status(cuda_ok):
+    # two groups over the same 1000 tokens hold more chunks than the scratch's chunk table
+    # allows: the kernels stay in bounds and record the error in the scratch header, which
+    # lh_noalloc_status reads; the next valid call clears it
+    import scale_calibration_b200 as lh
+    layer = synth.make_layer(8, 128, 1000, seed=32)
+    _, X, _ = gu.to_device(layer)
+    off = torch.tensor([0, 1000, 0, 1000], dtype=torch.int64, device="cuda")
+    H = torch.zeros(3, 8, 16, 16, device="cuda")
+    lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, 1000, 128, 128, off, 3, H)
+    assert lh.lh_noalloc_status() == 1  # LH_ERR_INVALID_ARG
+    assert "overlap" in lh.lh_last_error_message()
+    H1 = torch.zeros(1, 8, 16, 16, device="cuda")
+    lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, 1000, 128, 128, None, 1, H1)
+    assert lh.lh_noalloc_status() == 0
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
