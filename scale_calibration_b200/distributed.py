@@ -6,7 +6,8 @@ Local-Hessian: åŸºäºå±€éƒ¨ Hessian çš„ NVFP4 é€å—æƒé‡ç¼©æ”¾ç®—æ³•å®æˆ˜æŒ‡å
 tokens it holds and one all-reduce (sum) gives every rank the layer's H. The
 pages note that the Hessian is not synchronised across data-parallel ranks
 there; this module is that synchronisation. The sweep then needs no exchange:
-each rank sweeps a contiguous share of the rows with the full H.
+each rank sweeps its share of the blocks with the summed H (whole matrices of
+an expert bank, else a range of block columns; see sweep_shard).
 
 Plumbing only: the arithmetic runs in liblh.so (lh_accumulate_hessian,
 lh_sweep_scales, lh_fake_quant); torch.distributed (NCCL between GPUs) carries
@@ -37,6 +38,24 @@ def row_shard(c_out: int, rank: int, world: int):
     if world < 1 or not 0 <= rank < world:
         raise ValueError(f"rank {rank} out of range for world size {world}")
     return c_out * rank // world, c_out * (rank + 1) // world
+
+
+def sweep_shard(n_mats: int, c_out: int, J: int, rank: int, world: int):
+    """This rank's share of the sweep and fake-quant, as (kind, lo, hi):
+    ("mats", m0, m1): whole matrices [m0, m1) when there are at least as many
+    matrices as ranks (an expert bank: W, H and the global amax of a share are
+    contiguous, and each matrix's amax needs no exchange); ("cols", j0, j1): the
+    block columns [j0, j1) of every row of a single matrix (H + j0 blocks is
+    contiguous, and each rank keeps whole row tiles); ("rows", r0, r1) otherwise.
+    Every rank gets a share of about the same number of blocks; a share may be
+    empty when there are fewer units than ranks."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} out of range for world size {world}")
+    if n_mats >= world:
+        return "mats", n_mats * rank // world, n_mats * (rank + 1) // world
+    if n_mats == 1:
+        return "cols", J * rank // world, J * (rank + 1) // world
+    return ("rows",) + row_shard(c_out, rank, world)
 
 
 def allreduce_hessian(H, group=None):

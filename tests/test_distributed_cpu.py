@@ -97,3 +97,26 @@ def test_token_and_row_shares_partition(world):
     assert sum(lhd.row_shard(77, r, world)[1] - lhd.row_shard(77, r, world)[0] for r in range(world)) == 77
     with pytest.raises(ValueError):
         lhd.token_shard(10, world, world)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+@pytest.mark.parametrize("shape", [(1, 4096, 256), (64, 1536, 128), (1, 64, 8), (3, 40, 4)])
+def test_sweep_shares_cover_every_block_once(world, shape):
+    from scale_calibration_b200 import distributed as lhd
+    n_mats, c_out, J = shape
+    seen = np.zeros((n_mats, c_out, J), np.int64)
+    sizes = []
+    for r in range(world):
+        kind, lo, hi = lhd.sweep_shard(n_mats, c_out, J, r, world)
+        if kind == "mats":
+            seen[lo:hi] += 1
+            assert n_mats >= world
+        elif kind == "cols":
+            seen[:, :, lo:hi] += 1
+            assert n_mats == 1
+        else:
+            seen[:, lo:hi] += 1
+        sizes.append(int(seen.sum()) - sum(sizes))
+    assert np.all(seen == 1)
+    unit = {"mats": c_out * J, "cols": c_out, "rows": n_mats * J}[kind]
+    assert max(sizes) - min(sizes) <= unit   # shares differ by at most one unit

@@ -1,8 +1,9 @@
 """The N>1 plumbing of bench.py on CPU with gloo, world size 2.
 
-Each rank calibrates its own layer with no data-path collective; the only
-cross-rank traffic is the barrier and the max over ranks of the timed
-region. The reference arm runs on rank 0 alone and the other ranks exit 0.
+The timed region's end is the max over ranks; `--gpus N` without a launcher
+starts N local ranks; the reference arm runs on rank 0 alone and the other
+ranks exit 0. (The GPU arm's sharded step, with its NCCL all-reduces, needs
+GPUs; its share arithmetic is tested in test_distributed_cpu.py.)
 """
 import json
 import os
@@ -62,3 +63,18 @@ def test_reference_arm_runs_on_rank0_only():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_starts_its_own_ranks_for_gpus_n():
+    # `bench.py --gpus 2` with no launcher around it starts two local ranks itself
+    # (torch.distributed.run on 127.0.0.1); on the reference arm rank 0 prints the one line
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1",
+           "--warmup", "1", "--config", "0"]
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["impl"] == "reference" and d["extrapolated"] is True
+    assert "all-reduce" in d["config"]["parallelism"] and d["config"]["blocks"] == 512
