@@ -252,6 +252,28 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- CUDA path
+def fma_probe(lh, torch, dev, stream) -> dict:
+    """Measured FP32 FMA throughput on every SM, scalar (fma.rn.f32) and packed
+    (fma.rn.f32x2), with the library's probe kernel (CUDA events, best of 3)."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    out = torch.zeros(1, device=dev)
+    blocks, iters = 8 * sms, 4000
+    res = dict(blocks=blocks, iters=iters)
+    for name, packed in (("scalar_tflops", False), ("packed_tflops", True)):
+        for _ in range(2):
+            lh.lh_probe_fma(packed, blocks, iters, out, stream.cuda_stream)
+        ts = []
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lh.lh_probe_fma(packed, blocks, iters, out, stream.cuda_stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        res[name] = lh.lh_probe_fma_flop(blocks, iters) / min(ts) / 1e12
+    return res
+
+
 def make_share(layer, rank: int, ws: int) -> dict:
     """This rank's inputs: a contiguous token share (with its group offsets) for
     the Hessian and a share of the blocks for the sweep (see sweep_shard)."""
@@ -529,7 +551,10 @@ def run_ours(args):
     # ---- rooflines (this rank's share: the whole layer at one GPU)
     peaks = load_peaks()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    fp32_peak = sms * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s
+    probe = fma_probe(lh, torch, dev, stream)
+    # packed two-lane FMAs count twice when the probe shows they retire at twice the scalar rate
+    fma_width = 2 if probe["packed_tflops"] > 1.5 * probe["scalar_tflops"] else 1
+    fp32_peak = sms * FP32_LANES_PER_SM * 2 * fma_width * peaks["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s
     sweep_tflops = SWEEP_FLOP_PER_BLOCK * s_blocks / (t_sweep / 1e3) / 1e12 if t_sweep > 0 else 0.0
     hess_bytes = 2 * c_in * n_loc
     hess_gbs = hess_bytes / (t_hess / 1e3) / 1e9 if t_hess > 0 else 0.0
@@ -540,8 +565,9 @@ def run_ours(args):
                                              f"sweep_kernel_{layer.name}.md") if full else None,
                     traffic_note="DRAM bytes per launch from the committed ncu summary of this layer (null if the "
                                  "kernel changed since, or none was taken)",
-                    peak_note=f"FP32 CUDA-core peak {sms} SMs x 128 lanes x 2 flop x {peaks['sm_max_mhz']:.0f} MHz",
-                    flop_per_block=SWEEP_FLOP_PER_BLOCK, blocks_per_launch=int(s_blocks))
+                    peak_note=(f"FP32 CUDA-core peak {sms} SMs x 128 lanes x 2 flop x {fma_width} (FMAs per lane per "
+                               f"cycle, from the probe) x {peaks['sm_max_mhz']:.0f} MHz"),
+                    fma_probe=probe, flop_per_block=SWEEP_FLOP_PER_BLOCK, blocks_per_launch=int(s_blocks))
     if clocks.get("sm_mhz"):
         roofline["frac_at_measured_clock"] = sweep_tflops / (fp32_peak * clocks["sm_mhz"] / peaks["sm_max_mhz"])
     hessian = dict(tokens_per_s=n_loc / (t_hess / 1e3) if t_hess > 0 else None, bound="hbm",

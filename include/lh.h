@@ -120,6 +120,18 @@ LH_API lh_status lh_workspace_status(const void* workspace, void* stream);
 LH_API lh_status lh_debug_wait_timeout(void* workspace, size_t workspace_bytes, int64_t timeout_us, int arrive,
                                        void* stream);
 
+/* Diagnostics; the pages have no counterpart. FP32 FMA throughput probe for
+ * the sweep's roofline: launches `blocks` CTAs of 256 threads on `stream`, each
+ * thread running `iters` steps of 64 FMAs over 16 independent accumulators, as
+ * 32 packed two-lane FMAs (fma.rn.f32x2, packed != 0) or 64 scalar fma.rn.f32.
+ * The caller times
+ * the launch (CUDA events on `stream`); lh_probe_fma_flop(blocks, iters) is the
+ * flop count of one launch (2 per FMA). out: device, >= 1 float, never written
+ * in practice (it keeps the arithmetic from being removed).
+ * LH_ERR_INVALID_ARG: null out, blocks outside [1, 2^20], iters outside [1, 2^24]. */
+LH_API int64_t lh_probe_fma_flop(int64_t blocks, int64_t iters);
+LH_API lh_status lh_probe_fma(int packed, int64_t blocks, int64_t iters, float* out, void* stream);
+
 /* ------------------------------------------------------------------------
  * Allocation-free variant of lh_accumulate_hessian. The pages have no
  * counterpart: this is a library convenience for callers that cannot

@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     lh_accumulate_hessian_noalloc, lh_noalloc_status, lh_debug_wait_timeout, lh_hessian_workspace_bytes, lh_last_error_message, lh_status_string,
     lh_quantize_nvfp4, lh_sweep_scales, lh_workspace_status, lh_baseline_scales, LH_SCALE_MAX,
     LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE, lh_search_amax, lh_sweep_scales_ws, lh_sweep_workspace_bytes,
+    lh_probe_fma, lh_probe_fma_flop,
 )
 
 

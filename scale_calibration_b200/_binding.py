@@ -20,7 +20,7 @@ EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
     "lh_accumulate_hessian_noalloc", "lh_noalloc_status", "lh_debug_wait_timeout", "lh_quantize_nvfp4", "lh_baseline_scales",
-    "lh_search_amax", "lh_sweep_workspace_bytes", "lh_sweep_scales_ws",
+    "lh_search_amax", "lh_sweep_workspace_bytes", "lh_sweep_scales_ws", "lh_probe_fma", "lh_probe_fma_flop",
 ]
 LH_SCALE_MAX, LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE = range(3)
 
@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
         "lh_quantize_nvfp4": (I32, [P, I32, I64, I64, I64, I64, P, P, P, P, P, P, I32, P]),
         "lh_baseline_scales": (I32, [P, I32, I64, I64, I64, I64, P, I32, P, P, P]),
         "lh_search_amax": (I32, [P, I32, I64, I64, I64, I64, P, P, ctypes.c_double, ctypes.c_double, I64, P, P, P]),
+        "lh_probe_fma_flop": (I64, [I64, I64]),
+        "lh_probe_fma": (I32, [I32, I64, I64, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -149,6 +151,18 @@ def lh_debug_wait_timeout(workspace, workspace_bytes, timeout_us, arrive, stream
 
 def lh_workspace_status(workspace, stream=None) -> int:
     return _lib.lh_workspace_status(_ptr(workspace), _stream(stream))
+
+
+def lh_probe_fma_flop(blocks: int, iters: int) -> int:
+    return _lib.lh_probe_fma_flop(blocks, iters)
+
+
+def lh_probe_fma(packed: bool, blocks: int, iters: int, out, stream=None, check=True) -> int:
+    """FP32 FMA throughput probe (diagnostics): time the launch with CUDA events."""
+    s = _lib.lh_probe_fma(1 if packed else 0, blocks, iters, _ptr(out), _stream(stream))
+    if check:
+        _check(s, "lh_probe_fma")
+    return s
 
 
 def lh_noalloc_status(stream=None) -> int:

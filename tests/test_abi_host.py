@@ -189,3 +189,11 @@ def test_search_amax_rejects_bad_arguments():
         assert lh.lh_search_amax(**dict(ok, **over)) == want, over
         assert lh.lh_last_error_message() != ""
     assert lh.lh_search_amax(**dict(ok, c_out=0)) == 0
+
+
+def test_fma_probe_rejects_bad_arguments():
+    lh = _lh()
+    assert lh.lh_probe_fma_flop(148, 1000) == 148 * 256 * 1000 * 128
+    assert lh.lh_probe_fma_flop(0, 10) == 0
+    for packed, blocks, iters, out in [(1, 0, 10, FAKE), (0, 10, 0, FAKE), (1, 10, 10, 0), (0, 1 << 21, 10, FAKE)]:
+        assert lh.lh_probe_fma(packed, blocks, iters, out, stream=0, check=False) == 1
