@@ -84,17 +84,24 @@ LH_API lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, int6
  * offsets: device int64 [n_groups+1], non-decreasing, with the token range of
  *   each group (one per matrix / expert: tokens [offsets[g], offsets[g+1])), or
  *   NULL for a single group of all tokens (n_groups must then be 1). Offsets
- *   are clamped to [0, n_tokens_total] and empty or inverted ranges count as
- *   empty. Decreasing offsets whose ranges overlap by more than the workspace
- *   bound allows make the call record LH_ERR_INVALID_ARG in the workspace
- *   (see lh_workspace_status); H is then unspecified.
+ *   are clamped to [0, n_tokens_total]; tokens outside [offsets[0],
+ *   offsets[n_groups]) belong to no group. Decreasing offsets make the call
+ *   record LH_ERR_INVALID_ARG in the workspace (see lh_workspace_status); the
+ *   kernel stays in bounds and H is then unspecified.
  * H: device f32 [n_groups][c_in/16][16][16], read and written (H += ...):
  *   accumulation can be split over batches and resumed across calls.
  * workspace: device, at least lh_hessian_workspace_bytes(...) bytes, 256-byte
- *   aligned, owned by the caller; it holds the chunk table and per-chunk
- *   partial sums and must not be shared by calls in flight at the same time.
+ *   aligned, owned by the caller; it holds a status word, per-CTA counters and
+ *   the partial sums of the (slab, group) segments that several CTAs share.
+ *   Its size depends on n_tokens_total and c_in only, is at most about 5.3 MB,
+ *   and its contents need no clearing between calls; it must not be shared by
+ *   calls in flight at the same time.
+ * Work split: one kernel launch; each CTA (two per SM) reads an equal share of
+ *   X whatever the group sizes.
  * Numerics: bf16 products are exact in FP32; tensor-core FP32 accumulation
- *   over at most 128 tokens, then FP64 accumulation and one final rounding.
+ *   over at most 128 tokens, then FP64 accumulation, FP32 partial sums where a
+ *   segment spans several CTAs, summed in a fixed order (deterministic), and
+ *   one final rounding into H.
  * n_tokens_total == 0 is a no-op returning LH_OK.
  * ---------------------------------------------------------------------- */
 LH_API size_t lh_hessian_workspace_bytes(int64_t n_tokens_total, int64_t c_in, int64_t n_groups);
@@ -103,9 +110,11 @@ LH_API lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int64_t 
                                 int64_t ld_x, const int64_t* offsets, int64_t n_groups, float* H,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
-/* Status a kernel left in `workspace`: LH_OK, LH_ERR_TIMEOUT when a bounded
- * wait inside lh_accumulate_hessian gave up, or LH_ERR_INVALID_ARG when its
- * group offsets overlapped beyond the workspace bound. Synchronises `stream`. */
+/* Status the last launch on `workspace` left there: LH_OK, LH_ERR_TIMEOUT when
+ * a bounded wait inside lh_accumulate_hessian gave up, or LH_ERR_INVALID_ARG
+ * when its group offsets decreased. Synchronises `stream`. Each launch stamps
+ * the workspace with its own generation number, so an error of an earlier
+ * launch is not reported again. */
 LH_API lh_status lh_workspace_status(const void* workspace, void* stream);
 
 /* Diagnostics; the pages have no counterpart. Runs on `stream` the bounded
@@ -139,23 +148,23 @@ LH_API lh_status lh_probe_fma(int packed, int64_t blocks, int64_t iters, float* 
  * nearly all HBM for their own pools at start-up, plugins whose host owns
  * every device allocation, callers that avoid cudaMalloc/cudaFree because
  * those can synchronise the device). Same arguments and result as
- * lh_accumulate_hessian minus the workspace, which comes from a fixed 16 MiB
+ * lh_accumulate_hessian minus the workspace, which comes from a fixed 8 MiB
  * array compiled into the library; every GPU that loads the library holds it
  * until the process exits. Calls no cudaMalloc/cudaFree.
- *   - Returns LH_ERR_WORKSPACE, without launching, when
- *     lh_hessian_workspace_bytes(n_tokens_total, c_in, n_groups) > 16 MiB.
+ *   - The largest Hessian workspace is about 5.3 MB, so every size fits; a
+ *     size beyond the array would return LH_ERR_WORKSPACE without launching.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - Argument errors are the same, checked in the same order, as those of
- *     lh_accumulate_hessian; the size limit is checked after them.
- *   - All calls share the array (it keeps the last call's contents; what must
- *     start at zero is cleared by each call). Calls whose kernels overlap on
- *     the GPU race on it: serialise them (one stream, one thread at a time).
- *   - Errors the kernels find (an expired bounded wait, overlapping group
- *     offsets) are written to the array's header, not returned: read them with
- *     lh_noalloc_status after the call, before the next allocation-free call on
- *     that device clears them.
+ *     lh_accumulate_hessian.
+ *   - All calls share the array (it keeps the last call's contents; nothing in
+ *     it needs clearing between calls). Calls whose kernels overlap on the GPU
+ *     race on it: serialise them (one stream, one thread at a time).
+ *   - Errors the kernel finds (an expired bounded wait, decreasing group
+ *     offsets) are written to the array's status word, not returned: read them
+ *     with lh_noalloc_status after the call, before the next allocation-free
+ *     call on that device.
  * ---------------------------------------------------------------------- */
 LH_API lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dtype, int64_t n_tokens_total,
                                                int64_t c_in, int64_t ld_x, const int64_t* offsets,

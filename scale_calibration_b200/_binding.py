@@ -134,7 +134,7 @@ def lh_accumulate_hessian(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_gro
 def lh_accumulate_hessian_noalloc(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H, stream=None,
                                   check=True) -> int:
     """lh_accumulate_hessian with the workspace taken from the library's own
-    fixed 16 MiB device array, for callers that cannot allocate device memory."""
+    fixed 8 MiB device array, for callers that cannot allocate device memory."""
     s = _lib.lh_accumulate_hessian_noalloc(_ptr(X), _dtype(x_dtype), n_tokens_total, c_in, ld_x, _ptr(offsets),
                                            n_groups, _ptr(H), _stream(stream))
     if check:

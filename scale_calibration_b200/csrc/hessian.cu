@@ -6,33 +6,48 @@
 // "入口 API 与校准流程", Phase 2, accumulates H = sum X^T X over the calibration
 // tokens; the kernel contract lays H out as [cin/16, 16, 16].
 //
-// Design (B200):
-//  * Work item = (token chunk, 128-channel slab). A persistent grid of two CTAs
-//    per SM walks the items; each CTA has a TMA producer warp, an MMA warp and
-//    four epilogue warps, and two CTAs per SM keep more loads in flight and fill
-//    each other's pipeline gaps.
-//  * The producer stages [128 tokens x 128 channels] bf16 tiles (two 64-channel
-//    TMA boxes, 128-byte swizzle) in a 3-deep shared-memory ring (96 KB).
-//  * The tile is channel-contiguous, so it is an MN-major operand for both
-//    A = tile^T (M = channels, K = tokens) and B = tile (K = tokens,
-//    N = channels): one tcgen05.mma (M = N = 128, K = 16, FP32 accumulate in
-//    TMEM) per 16 tokens forms the 128x128 Gram block of the slab, of which the
-//    8 diagonal 16x16 blocks are the local Hessians. The off-diagonal products
-//    cost tensor-core time only; the kernel stays bound by the HBM read of X.
-//  * Each stage accumulates into one of two TMEM buffers; the epilogue warps
-//    read the diagonal blocks (tcgen05.ld), free the buffer, and add them into
-//    FP64 registers, so FP32 accumulation never spans more than 128 tokens.
-//  * A chunk's sums go to the workspace; a second kernel adds the chunks of
-//    each group in a fixed order (FP64) into H. No atomics: the result is
-//    deterministic.
-//  * Ragged ends (group boundaries inside a tile) are masked by zeroing the
-//    token rows past the end inside the last 16-row MMA step; rows past the
-//    tensor end arrive as zeros from TMA.
+// Design (B200): one kernel launch per call, bound by the HBM read of X.
+//  * Work split: the tokens are cut into equal bands and the CTAs of the grid
+//    (about two per SM) form one team per band, one CTA per 128-channel slab
+//    (or per run of slabs when the layer is wider than the grid). The CTAs of a
+//    team start together on the same token rows and read them slab by slab,
+//    so the whole width of each row is fetched from HBM at about the same
+//    time, and every CTA reads the same number of bytes whatever the group
+//    sizes. A CTA walks its band as pieces (one group's run of tokens) cut
+//    into stages of at most 128 tokens that never cross a group's end.
+//  * Per CTA: a TMA producer warp, an MMA warp and four epilogue warps. The
+//    producer stages [tokens x 128 channels] bf16 tiles (two 64-channel boxes,
+//    128-byte swizzle; 128-token boxes, or 16-token boxes for the short last
+//    stage of a piece) in a 3-deep shared-memory ring. The tile is
+//    channel-contiguous, so it is an MN-major operand for both A = tile^T and
+//    B = tile: one tcgen05.mma (M = N = 128, K = 16, FP32 accumulate in TMEM)
+//    per 16 tokens forms the 128x128 Gram block of the slab, of which the 8
+//    diagonal 16x16 blocks are the local Hessians (the off-diagonal products
+//    cost tensor-core time only). Token rows of the last 16-row step that lie
+//    past the piece are zeroed in shared memory before the MMA.
+//  * The epilogue warps read each stage's 8 diagonal blocks from one of two
+//    TMEM buffers (tcgen05.ld) and add them into FP64 registers, so FP32
+//    accumulation never spans more than 128 tokens. At the end of a piece:
+//    if the group's tokens of that slab lie in this CTA's band alone, the CTA
+//    is the only one to add to those entries of H and adds its sum with
+//    vector reductions (red.global.add.v4.f32, no wait for H to load);
+//    otherwise it stores the sum as its part of the (slab, group) segment in
+//    the workspace. A second kernel, launched as a programmatic dependent,
+//    adds each split segment's parts in band order to H. The order of every
+//    sum is fixed, so H is deterministic; no CTA waits on another.
+//  * Nothing in the workspace needs clearing between calls: the parts are
+//    written before they are read in every call, and the status word carries
+//    the call's 48-bit generation, so a stale value from an earlier call (or a
+//    fresh buffer) never matches it.
 //  * Every mbarrier wait is bounded (1 s of globaltimer); on expiry the kernel
-//    records LH_ERR_TIMEOUT in the workspace header and the CTA winds down.
+//    records LH_ERR_TIMEOUT in the workspace status word and the CTA winds
+//    down. Decreasing group offsets are recorded as LH_ERR_INVALID_ARG (the
+//    walk stays in bounds).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+#include <chrono>
 #include <mutex>
 
 #include "common.cuh"
@@ -41,16 +56,18 @@
 namespace lh {
 namespace {
 
-constexpr int kSlab = 128;                       // channels per item = MMA M = N
-constexpr int kStageTok = 128;                   // tokens per pipeline stage
+constexpr int kSlab = 128;                       // channels per slab = MMA M = N
+constexpr int kStageTok = 128;                   // tokens per full pipeline stage
+constexpr int kSmallBox = 16;                    // token rows of the boxes for a short stage
 constexpr int kStages = 3;
-constexpr int kHalfBytes = kStageTok * 64 * 2;   // one 64-channel TMA box: 16 KB
+constexpr int kHalfBytes = kStageTok * 64 * 2;   // one 128-token, 64-channel TMA box: 16 KB
 constexpr int kStageBytes = 2 * kHalfBytes;      // 32 KB
 constexpr int kThreads = 192;                    // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kTmemCols = 256;                   // two 128x128 FP32 accumulators
-constexpr int kMinItems = 256;                   // work items wanted for one launch
-constexpr int kMaxItems = 16384;
+constexpr int kMaxCtas = 320;                    // grid bound (two CTAs per SM, up to 160 SMs)
 constexpr size_t kHeaderBytes = 256;
+constexpr int kPartFloats = 8 * 256;             // one slab's 8 blocks of 16x16, FP32
+constexpr unsigned long long kGenMask = (1ull << 48) - 1;
 
 // Instruction descriptor of tcgen05.mma kind::f16: D = F32, A = B = BF16,
 // both MN-major, N = 128, M = 128.
@@ -62,25 +79,39 @@ constexpr uint32_t kIdesc = (1u << 4)            // D format F32
                             | ((uint32_t)(kSlab >> 3) << 17)   // N >> 3
                             | ((uint32_t)(kSlab >> 4) << 24);  // M >> 4
 
-struct Chunk {
-    int64_t start;
-    int32_t len;
-    int32_t group;
-};
 
+// The grid: `bands` teams of `sgroups` CTAs. With at most `cap` CTAs: one CTA
+// per slab and as many bands as fit (each at least one stage of tokens), or,
+// for layers with more slabs than CTAs, one band and runs of slabs.
+struct Grid {
+    int64_t slabs, sgroups, bands;
+    int64_t ctas() const { return sgroups * bands; }
+};
+constexpr Grid make_grid(int64_t n_tok, int64_t c_in, int64_t cap) {
+    Grid gr{};
+    gr.slabs = (c_in + kSlab - 1) / kSlab;
+    gr.sgroups = gr.slabs < cap ? gr.slabs : cap;
+    const int64_t by_cap = cap / gr.sgroups;
+    const int64_t by_tok = (n_tok + kStageTok - 1) / kStageTok;
+    gr.bands = by_cap < by_tok ? by_cap : by_tok;
+    if (gr.bands < 1) gr.bands = 1;
+    return gr;
+}
+
+// Workspace: [header: status word, generation of the last launch][parts:
+// [bands][slabs][2][8 blocks][16][16] FP32]. Parts exist only with several
+// bands (a layer no wider than the grid), so their count is bounded by twice
+// the grid size.
 struct WsLayout {
-    size_t table_off, kfirst_off, partial_off, total;
-    int64_t max_chunks;
+    size_t part_off, total;
 };
-
-struct Plan {
-    int64_t chunk;       // tokens per chunk (multiple of kStageTok)
-    int64_t n_slabs;
-    int64_t max_chunks;  // bound on the number of chunks
-    WsLayout ws;
-};
-
-inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+constexpr WsLayout ws_layout(const Grid& gr) {
+    WsLayout w{};
+    const size_t pairs = gr.bands > 1 ? (size_t)gr.bands * (size_t)gr.slabs : 0;
+    w.part_off = kHeaderBytes;
+    w.total = w.part_off + sizeof(float) * kPartFloats * 2 * pairs;
+    return w;
+}
 
 using namespace lh::tc;
 
@@ -96,11 +127,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
     d |= (uint64_t)2 << 61;                              // SWIZZLE_128B
     return d;
 }
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
-    mma_f16(tmem_d, a, b, kIdesc, accumulate);
-}
-__device__ __forceinline__ void tc_fence_before() { fence_before(); }
-__device__ __forceinline__ void tc_fence_after() { fence_after(); }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -113,215 +139,316 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-
-int64_t chunks_bound(int64_t n_tok, int64_t chunk, int64_t n_groups) {
-    return (n_tok + chunk - 1) / chunk + (n_groups - 1);
-}
-
-Plan make_plan(int64_t n_tok, int64_t c_in, int64_t n_groups) {
-    Plan p;
-    p.n_slabs = (c_in + kSlab - 1) / kSlab;
-    int64_t ch = 2048;
-    while (ch > kStageTok && chunks_bound(n_tok, ch, n_groups) * p.n_slabs < kMinItems) ch /= 2;
-    while (chunks_bound(n_tok, ch, n_groups) * p.n_slabs > kMaxItems && ch < ((int64_t)1 << 40)) ch *= 2;
-    p.chunk = ch;
-    p.max_chunks = chunks_bound(n_tok, ch, n_groups);
-    const int64_t J = c_in / 16;
-    p.ws.max_chunks = p.max_chunks;
-    p.ws.table_off = kHeaderBytes;
-    p.ws.kfirst_off = p.ws.table_off + align256(sizeof(Chunk) * (size_t)p.max_chunks);
-    p.ws.partial_off = p.ws.kfirst_off + align256(sizeof(int32_t) * (size_t)(n_groups + 1));
-    p.ws.total = p.ws.partial_off + sizeof(float) * 256 * (size_t)J * (size_t)p.max_chunks;
-    return p;
+// A bounded mbarrier wait taken by a whole warp, with one answer for all its lanes.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag));
 }
 
 struct KParams {
-    int64_t n_tok;
-    int64_t J;
-    int64_t n_slabs;
-    int64_t chunk;
-    int64_t n_items_max;
-    int grouped;
-    const Chunk* table;
-    const int32_t* n_chunks_dev;  // grouped: number of chunks (device)
-    float* partial;               // [max_chunks][J][256]
-    int* err;                     // workspace header word 0
+    int64_t N;           // tokens
+    int64_t J;           // block columns (c_in / 16)
+    int64_t G;           // groups (1 without offsets)
+    int64_t slabs, sgroups, bands;  // the grid: bands x sgroups CTAs (see Grid)
+    const int64_t* off;  // [G + 1] group offsets, or null: one group of all tokens
+    float* H;            // [G][J][16][16], H +=
+    unsigned long long* hdr;       // [0] status: gen << 16 | lh_status, written on error; [1] gen of the launch
+    float* parts;                  // [bands][slabs][2][8][16][16]
+    unsigned long long gen;        // this launch's generation, < 2^48
 };
 
-__device__ __forceinline__ bool item_chunk(const KParams& p, int64_t item, int64_t n_chunks, int64_t& k,
-                                           int64_t& sl, int64_t& start, int64_t& len) {
-    k = item / p.n_slabs;
-    sl = item - k * p.n_slabs;
-    if (k >= n_chunks) return false;
-    if (p.grouped) {
-        const Chunk c = p.table[k];
-        start = c.start;
-        len = c.len;
-    } else {
-        start = k * p.chunk;
-        len = min(p.chunk, p.n_tok - start);
-    }
-    return true;
+// First token of band k (the bands split [0, N) as evenly as integers allow).
+__device__ __forceinline__ int64_t band_start(const KParams& p, int64_t k) { return p.N * k / p.bands; }
+// The band holding token t.
+__device__ __forceinline__ int64_t band_of(const KParams& p, int64_t t) {
+    int64_t k = min(t * p.bands / p.N, p.bands - 1);
+    while (k + 1 < p.bands && band_start(p, k + 1) <= t) ++k;
+    while (k > 0 && band_start(p, k) > t) --k;
+    return k;
+}
+// Slot of band k's part of a segment that starts at token seg_lo: 0 when the
+// segment holds the band's first token (the band's first piece of the slab),
+// else 1 (its last piece: only the segment's first band).
+__device__ __forceinline__ int64_t part_slot(const KParams& p, int64_t k, int64_t slab, int64_t seg_lo) {
+    return (k * p.slabs + slab) * 2 + (seg_lo <= band_start(p, k) ? 0 : 1);
 }
 
+// Token range of group g, clamped to [0, N]; an inverted range is empty.
+__device__ __forceinline__ void group_range(const KParams& p, int64_t g, int64_t& lo, int64_t& hi) {
+    if (!p.off) { lo = 0; hi = p.N; return; }
+    lo = min(max(__ldg(p.off + g), (int64_t)0), p.N);
+    hi = min(max(__ldg(p.off + g + 1), lo), p.N);
+}
+
+// First group g whose offsets[g + 1] exceeds token t (G when none), by the whole
+// warp: each step probes 32 evenly spaced offsets at once (two steps for G <= 1024).
+// Exact for non-decreasing offsets; a bounded answer in [0, G] for any others.
+__device__ int64_t find_group(const KParams& p, int64_t t, int lane) {
+    if (!p.off) return 0;
+    int64_t lo = 0, n = p.G;
+    while (n > 32) {
+        const int64_t step = (n + 31) / 32;
+        const int64_t ak = min(lo + (int64_t)(lane + 1) * step - 1, lo + n - 1);
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, __ldg(p.off + ak + 1) > t);
+        if (m == 0) return lo + n;
+        const int k = __ffs(m) - 1;
+        const int64_t nlo = lo + (int64_t)k * step;
+        n = min(lo + (int64_t)(k + 1) * step - 1, lo + n - 1) - nlo + 1;
+        lo = nlo;
+    }
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, lane < n && __ldg(p.off + lo + lane + 1) > t);
+    return m ? lo + __ffs(m) - 1 : lo + n;
+}
+
+// One stage as the producer hands it to the MMA warp and, through it, to the
+// epilogue.
+struct StageDesc {
+    int32_t ntok;     // tokens of the stage (1..128); 0 marks the end of the CTA's work
+    int32_t flags;    // bit 0: last stage of its piece (flush)
+    int32_t slab;
+    int32_t g;
+    int64_t seg_lo;   // the group's first token (clamped): its segment in this slab is
+    int64_t seg_hi;   // [seg_lo, seg_hi)
+};
+
+struct Smem {
+    uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], dfull[2];
+    StageDesc sdesc[kStages];  // per ring slot, written before the slot's loads
+    StageDesc edesc[2];        // per TMEM buffer, for the epilogue
+    uint32_t tmem_slot;
+    int abort_flag;
+};
+
 __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                 const __grid_constant__ CUtensorMap tmap16,
                                                                  const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled tiles
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-    // bars: full[kStages], empty[kStages], tfull[2], tempty[2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 4);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    uint8_t* tiles_p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Smem& S = *reinterpret_cast<Smem*>(tiles_p + kStages * kStageBytes);
+    volatile int* abort_flag = &S.abort_flag;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const uint32_t tiles = smem_u32(smem);
-    auto full_bar = [&](int s) { return smem_u32(bars + s); };
-    auto empty_bar = [&](int s) { return smem_u32(bars + kStages + s); };
-    auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * kStages + a); };
-    auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * kStages + 2 + a); };
+    const uint32_t tiles = smem_u32(tiles_p);
+    const int64_t b = blockIdx.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
+            mbar_init(smem_u32(&S.full[s]), 1);
+            mbar_init(smem_u32(&S.empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(tfull_bar(a), 1);
-            mbar_init(tempty_bar(a), 4);
+            mbar_init(smem_u32(&S.tfull[a]), 1);
+            mbar_init(smem_u32(&S.tempty[a]), 4);
+            mbar_init(smem_u32(&S.dfull[a]), 1);
         }
-        *abort_flag = 0;
+        S.abort_flag = 0;
         mbar_init_fence();
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
+    if (warp == 1) tmem_alloc(smem_u32(&S.tmem_slot), kTmemCols);
+    fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-    // set-up above overlaps the kernel before (programmatic launch); X, the chunk table
-    // and the workspace header are read only after it has finished
+    fence_after();
+    const uint32_t tmem_base = S.tmem_slot;
+    // the set-up above overlaps the kernel before (programmatic launch); X, the
+    // offsets, H and the workspace are touched only after it has finished
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+    // the parts kernel may launch now: its CTAs wait on the device for this grid to finish
+    // (griddepcontrol.wait), so they start adding parts the moment the last CTA exits
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x == 0 && b == 0) p.hdr[1] = p.gen;
 
-    const int64_t n_chunks = p.grouped ? (int64_t)(*p.n_chunks_dev) : (p.n_tok + p.chunk - 1) / p.chunk;
+    const int64_t band = b / p.sgroups, sg = b - band * p.sgroups;
+    const int64_t bt0 = band_start(p, band), bt1 = band_start(p, band + 1);  // this CTA's tokens
+    const int64_t sl0 = p.slabs * sg / p.sgroups, sl1 = p.slabs * (sg + 1) / p.sgroups;  // and slabs
     bool ok = true;
 
     if (warp == 0) {
-        // ---------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int64_t item = blockIdx.x; ok && item < p.n_items_max; item += gridDim.x) {
-                int64_t k, sl, start, len;
-                if (!item_chunk(p, item, n_chunks, k, sl, start, len)) break;
-                const int n_st = (int)((len + kStageTok - 1) / kStageTok);
-                for (int st = 0; st < n_st; ++st) {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1, abort_flag)) { ok = false; break; }
-                    mbar_expect_tx(full_bar(stage), kStageBytes);
-                    const int y = (int)(start + (int64_t)st * kStageTok);
-                    const int x = (int)(sl * kSlab);
-                    tma_load_2d(tiles + stage * kStageBytes, &tmap, x, y, full_bar(stage));
-                    tma_load_2d(tiles + stage * kStageBytes + kHalfBytes, &tmap, x + 64, y, full_bar(stage));
+        // ------------------------------------------------------------ TMA producer
+        // The whole warp walks the band (group look-ups are warp-wide); lane 0 issues.
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap16)) : "memory");
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int64_t slab = sl0; ok && slab < sl1; ++slab) {
+            int64_t t = bt0;
+            int64_t g = find_group(p, t, lane);
+            while (ok && t < bt1) {
+                int64_t lo = 0, hi = 0;
+                while (g < p.G) {
+                    group_range(p, g, lo, hi);
+                    if (hi > t) break;
+                    ++g;
+                }
+                if (g >= p.G || lo >= bt1) break;  // no group holds the rest of the band
+                t = max(t, lo);
+                const int64_t t1 = min(hi, bt1);
+                for (int64_t ts = t; ts < t1; ts += kStageTok) {
+                    const int ntok = (int)min((int64_t)kStageTok, t1 - ts);
+                    if (!warp_wait(smem_u32(&S.empty[stage]), phase ^ 1, abort_flag)) { ok = false; break; }
+                    if (lane == 0) {
+                        StageDesc& d = S.sdesc[stage];
+                        d.ntok = ntok;
+                        d.flags = (ts + kStageTok >= t1) ? 1 : 0;
+                        d.slab = (int32_t)slab;
+                        d.g = (int32_t)g;
+                        d.seg_lo = lo;
+                        d.seg_hi = hi;
+                        const int x = (int)(slab * kSlab);
+                        const int y = (int)ts;
+                        const uint32_t dst = tiles + stage * kStageBytes;
+                        const uint32_t fb = smem_u32(&S.full[stage]);
+                        if (ntok == kStageTok) {
+                            mbar_expect_tx(fb, kStageBytes);
+                            tma_load_2d(dst, &tmap, x, y, fb);
+                            tma_load_2d(dst + kHalfBytes, &tmap, x + 64, y, fb);
+                        } else {
+                            // the short last stage of a piece: only the 16-row boxes it needs
+                            const int nb = (ntok + kSmallBox - 1) / kSmallBox;
+                            mbar_expect_tx(fb, (uint32_t)(nb * 2 * kSmallBox * 128));
+                            for (int i = 0; i < nb; ++i) {
+                                tma_load_2d(dst + i * kSmallBox * 128, &tmap16, x, y + i * kSmallBox, fb);
+                                tma_load_2d(dst + kHalfBytes + i * kSmallBox * 128, &tmap16, x + 64,
+                                            y + i * kSmallBox, fb);
+                            }
+                        }
+                    }
+                    __syncwarp();
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
+                t = t1;
+            }
+        }
+        if (ok) {
+            // end marker for the MMA warp: a stage of 0 tokens
+            if (warp_wait(smem_u32(&S.empty[stage]), phase ^ 1, abort_flag)) {
+                if (lane == 0) {
+                    S.sdesc[stage].ntok = 0;
+                    mbar_arrive(smem_u32(&S.full[stage]));
+                }
+            } else {
+                ok = false;
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
+        // ------------------------------------------------------------ MMA issuer
         int stage = 0;
         uint32_t phase = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int64_t item = blockIdx.x; ok && item < p.n_items_max; item += gridDim.x) {
-            int64_t k, sl, start, len;
-            if (!item_chunk(p, item, n_chunks, k, sl, start, len)) break;
-            const int n_st = (int)((len + kStageTok - 1) / kStageTok);
-            for (int st = 0; st < n_st; ++st) {
-                if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
-                const int nv = (int)min((int64_t)kStageTok, len - (int64_t)st * kStageTok);
-                const int ksteps = (nv + 15) >> 4;
-                const int pad_end = ksteps * 16;
-                if (nv < pad_end) {
-                    // zero token rows [nv, pad_end) of both 64-channel halves (128 bytes each)
-                    uint8_t* base = smem + stage * kStageBytes;
-                    const int n16 = (pad_end - nv) * 8;  // 16-byte chunks per half
-                    for (int i = lane; i < 2 * n16; i += 32) {
-                        const int h = i / n16, rem = i - h * n16;
-                        const int row = nv + (rem >> 3), c = rem & 7;
-                        *reinterpret_cast<uint4*>(base + h * kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                    }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                }
-                __syncwarp();
-                if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1, abort_flag)) { ok = false; break; }
-                tc_fence_after();
+        while (ok) {
+            if (!warp_wait(smem_u32(&S.full[stage]), phase, abort_flag)) { ok = false; break; }
+            const StageDesc d = S.sdesc[stage];
+            // the stage (or the end marker) goes to the epilogue with a free TMEM buffer
+            if (!warp_wait(smem_u32(&S.tempty[acc]), acc_phase ^ 1, abort_flag)) { ok = false; break; }
+            if (d.ntok == 0) {
                 if (lane == 0) {
-                    const uint32_t a0 = tiles + stage * kStageBytes;
-                    for (int kk = 0; kk < ksteps; ++kk) {
-                        const uint64_t d = smem_desc(a0 + kk * 2048);  // 16 token rows of 128 bytes
-                        mma_bf16(tmem_base + acc * kSlab, d, d, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(empty_bar(stage));
-                    mma_commit(tfull_bar(acc));
+                    S.edesc[acc] = d;
+                    mbar_arrive(smem_u32(&S.dfull[acc]));
                 }
-                __syncwarp();
-                if (++stage == kStages) { stage = 0; phase ^= 1; }
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1;
+                break;
             }
+            const int ksteps = (d.ntok + 15) >> 4;
+            const int pad_end = ksteps * 16;
+            if (d.ntok < pad_end) {
+                // zero token rows [ntok, pad_end) of both 64-channel halves (128 bytes each)
+                uint8_t* base = tiles_p + stage * kStageBytes;
+                const int n16 = (pad_end - d.ntok) * 8;  // 16-byte chunks per half
+                for (int i = lane; i < 2 * n16; i += 32) {
+                    const int h = i / n16, rem = i - h * n16;
+                    const int row = d.ntok + (rem >> 3), c = rem & 7;
+                    *reinterpret_cast<uint4*>(base + h * kHalfBytes + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async();
+            }
+            __syncwarp();
+            fence_after();
+            if (lane == 0) {
+                S.edesc[acc] = d;
+                mbar_arrive(smem_u32(&S.dfull[acc]));
+                const uint32_t a0 = tiles + stage * kStageBytes;
+                for (int kk = 0; kk < ksteps; ++kk) {
+                    const uint64_t sd = smem_desc(a0 + kk * 2048);  // 16 token rows of 128 bytes
+                    mma_f16(tmem_base + acc * kSlab, sd, sd, kIdesc, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&S.empty[stage]));
+                mma_commit(smem_u32(&S.tfull[acc]));
+            }
+            __syncwarp();
+            if (++stage == kStages) { stage = 0; phase ^= 1; }
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
         }
     } else {
-        // ---------------------------------------------------------- epilogue
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 64;    // 0..127
         const int q = warp & 3;              // TMEM lane quarter this warp may access
         const int row = 32 * q + lane;       // channel within the slab
         const int blk = row >> 4, a = row & 15;
-        const bool hi = lane >= 16;
+        const bool hi16 = lane >= 16;
+        // this CTA's slice of the offsets: no adjacent pair may decrease
+        if (p.off) {
+            const int64_t nct = p.bands * p.sgroups;
+            const int64_t g0 = p.G * b / nct, g1 = p.G * (b + 1) / nct;
+            bool bad = false;
+            for (int64_t g = g0 + et; g < g1; g += 128) bad |= __ldg(p.off + g + 1) < __ldg(p.off + g);
+            if (bad) atomicExch(p.hdr, (p.gen << 16) | (unsigned long long)LH_ERR_INVALID_ARG);
+        }
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int64_t item = blockIdx.x; ok && item < p.n_items_max; item += gridDim.x) {
-            int64_t k, sl, start, len;
-            if (!item_chunk(p, item, n_chunks, k, sl, start, len)) break;
-            const int n_st = (int)((len + kStageTok - 1) / kStageTok);
-            double sum[16];
+        double sum[16];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) sum[c] = 0.0;
-            for (int st = 0; st < n_st; ++st) {
-                if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                uint32_t r[32];
-                tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + acc * kSlab + 32 * q, r);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(tempty_bar(acc));
+        for (int c = 0; c < 16; ++c) sum[c] = 0.0;
+        while (ok) {
+            if (!warp_wait(smem_u32(&S.dfull[acc]), acc_phase, abort_flag)) { ok = false; break; }
+            const StageDesc d = S.edesc[acc];
+            if (d.ntok == 0) break;
+            if (!warp_wait(smem_u32(&S.tfull[acc]), acc_phase, abort_flag)) { ok = false; break; }
+            fence_after();
+            uint32_t r[32];
+            tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + acc * kSlab + 32 * q, r);
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&S.tempty[acc]));
 #pragma unroll
-                for (int c = 0; c < 16; ++c) sum[c] += (double)__uint_as_float(hi ? r[16 + c] : r[c]);
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1;
-            }
-            if (!ok) break;
-            const int64_t jb = sl * 8 + blk;
-            if (jb < p.J) {
-                float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)k * p.J + jb) * 256 + a * 16);
+            for (int c = 0; c < 16; ++c) sum[c] += (double)__uint_as_float(hi16 ? r[16 + c] : r[c]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+            if (!(d.flags & 1)) continue;
+
+            // ---- end of a piece: add it to H, alone or through the parts
+            const int64_t jb = (int64_t)d.slab * 8 + blk;
+            const bool in_h = jb < p.J;
+            float* hrow = p.H + (((int64_t)d.g * p.J + jb) * 16 + a) * 16;
+            if (d.seg_lo >= bt0 && d.seg_hi <= bt1) {
+                // the group's tokens of this slab are all in this band: no other CTA adds to
+                // these entries of H, so a reduction is one ordered addition, H = fp32(H + fp32(sum))
+                if (in_h) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(hrow + 4 * c),
+                                     "f"((float)sum[4 * c]), "f"((float)sum[4 * c + 1]), "f"((float)sum[4 * c + 2]),
+                                     "f"((float)sum[4 * c + 3])
+                                     : "memory");
+                }
+            } else {
+                // this band's part of a segment that several bands share; the parts kernel adds them
+                float4* part = reinterpret_cast<float4*>(p.parts + part_slot(p, band, d.slab, d.seg_lo) * kPartFloats +
+                                                         row * 16);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    dst[c] = make_float4((float)sum[4 * c], (float)sum[4 * c + 1], (float)sum[4 * c + 2],
-                                         (float)sum[4 * c + 3]);
+                    __stcg(part + c, make_float4((float)sum[4 * c], (float)sum[4 * c + 1], (float)sum[4 * c + 2],
+                                                 (float)sum[4 * c + 3]));
             }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) sum[c] = 0.0;
         }
     }
 
     if (!ok) {
         *abort_flag = 1;
-        atomicExch(p.err, (int)LH_ERR_TIMEOUT);
+        atomicExch(p.hdr, (p.gen << 16) | (unsigned long long)LH_ERR_TIMEOUT);
     }
-    // the reduction may launch now; it waits for this grid to finish before reading
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
     if (*abort_flag) {
         // let copies and MMAs already issued by this CTA land before leaving
@@ -329,21 +456,75 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
         while (global_ns() - t0 < 200000ull) {
         }
     }
-    tc_fence_after();
-    if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
-                     : "memory");
-    }
+    fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
-// Diagnostics: the bounded wait of the kernels above, on an mbarrier that
+// Adds the parts of every segment that several bands share to H. CTA (slab, k)
+// looks at band boundary k of one slab: the group holding tokens t_k - 1 and
+// t_k (t_k the first token of band k) crosses it; the CTA of the segment's
+// first crossing (the group starts in band k - 1) adds the parts of bands
+// k - 1 .. b1 in band order, four H entries per thread with up to eight parts'
+// loads in flight. Launched as a programmatic dependent of hessian_tc_kernel:
+// its CTAs wait for that grid to finish before reading.
+constexpr int kPartsThreads = 512;  // 128 rows x 4 column chunks of a slab
+__global__ void __launch_bounds__(kPartsThreads) hessian_parts_kernel(const KParams p) {
+    __shared__ int64_t s_lo, s_hi, s_g;
+    const int64_t slab = blockIdx.x;  // boundary 1 of every slab first: with one group, the only ones at work
+    const int64_t k = blockIdx.y + 1;
+    const int64_t tk = band_start(p, k);
+    const int lane = threadIdx.x & 31;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x < 32) {
+        // the same walk as the producer's: the first group that holds token tk - 1
+        int64_t g = find_group(p, tk - 1, lane), lo = 0, hi = 0;
+        while (g < p.G) {
+            group_range(p, g, lo, hi);
+            if (hi > tk - 1) break;
+            ++g;
+        }
+        if (lane == 0) {
+            s_g = g;
+            s_lo = lo;
+            s_hi = hi;
+        }
+    }
+    __syncthreads();
+    const int64_t g = s_g, lo = s_lo, hi = s_hi;
+    // a segment that crosses boundary k and starts in band k - 1
+    if (g >= p.G || lo >= tk || hi <= tk || lo < band_start(p, k - 1)) return;
+    const int row = threadIdx.x >> 2, c4 = threadIdx.x & 3;
+    const int64_t jb = slab * 8 + (row >> 4);
+    if (jb >= p.J) return;
+    const int64_t b1 = band_of(p, hi - 1);
+    float4* h4 = reinterpret_cast<float4*>(p.H + ((g * p.J + jb) * 16 + (row & 15)) * 16) + c4;
+    const float4 h0 = *h4;
+    double t0 = h0.x, t1 = h0.y, t2 = h0.z, t3 = h0.w;
+    for (int64_t k0 = k - 1; k0 <= b1; k0 += 8) {
+        float4 v[8];  // eight parts' loads in flight, then added in band order
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (k0 + i <= b1)
+                v[i] = __ldcg(reinterpret_cast<const float4*>(p.parts + part_slot(p, k0 + i, slab, lo) * kPartFloats +
+                                                              row * 16) + c4);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (k0 + i <= b1) {
+                t0 += v[i].x; t1 += v[i].y; t2 += v[i].z; t3 += v[i].w;
+            }
+    }
+    *h4 = make_float4((float)t0, (float)t1, (float)t2, (float)t3);
+}
+
+// Diagnostics: the bounded wait of the kernel above, on an mbarrier that
 // nothing arrives on (arrive == 0) or that thread 0 completes first
 // (arrive != 0); a wait that runs out records LH_ERR_TIMEOUT in the workspace
-// header like hessian_tc_kernel does.
-__global__ void wait_timeout_kernel(int* err, uint64_t timeout_ns, int arrive) {
+// header as hessian_tc_kernel does.
+__global__ void wait_timeout_kernel(unsigned long long* hdr, unsigned long long gen, uint64_t timeout_ns, int arrive) {
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
     if (threadIdx.x == 0) {
+        hdr[1] = gen;
         mbar_init(smem_u32(&bar), 1);
         abort_flag = 0;
         mbar_init_fence();
@@ -351,113 +532,20 @@ __global__ void wait_timeout_kernel(int* err, uint64_t timeout_ns, int arrive) {
     __syncthreads();
     if (arrive && threadIdx.x == 0) mbar_arrive(smem_u32(&bar));
     const bool ok = mbar_wait(smem_u32(&bar), 0u, &abort_flag, timeout_ns);
-    if (!ok) atomicExch(err, (int)LH_ERR_TIMEOUT);
+    if (!ok) atomicExch(hdr, (gen << 16) | (unsigned long long)LH_ERR_TIMEOUT);
 }
 
-// Builds the chunk table of the grouped case: each group's token range split
-// into chunks of `chunk` tokens; kfirst[g] = first chunk of group g.
-__global__ void chunk_table_kernel(const int64_t* __restrict__ offsets, int64_t G, int64_t n_tok, int64_t chunk,
-                                   int64_t max_chunks, Chunk* __restrict__ table, int32_t* __restrict__ kfirst,
-                                   int32_t* __restrict__ n_chunks_out, int* __restrict__ status) {
-    __shared__ int64_t scan[1024];
-    __shared__ int64_t base_s;
-    const int tid = threadIdx.x;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the main kernel may set up meanwhile
-    if (tid == 0) base_s = 0;
-    __syncthreads();
-    for (int64_t g0 = 0; g0 < G; g0 += blockDim.x) {
-        const int64_t g = g0 + tid;
-        int64_t lo = 0, hi = 0, cnt = 0;
-        if (g < G) {
-            lo = min(max(offsets[g], (int64_t)0), n_tok);
-            hi = min(max(offsets[g + 1], lo), n_tok);
-            cnt = (hi - lo + chunk - 1) / chunk;
-        }
-        scan[tid] = cnt;
-        __syncthreads();
-        for (int off = 1; off < (int)blockDim.x; off <<= 1) {  // inclusive Hillis-Steele scan
-            const int64_t v = tid >= off ? scan[tid - off] : 0;
-            __syncthreads();
-            scan[tid] += v;
-            __syncthreads();
-        }
-        const int64_t base = base_s;
-        const int64_t first = base + scan[tid] - cnt;
-        if (g < G) {
-            kfirst[g] = (int32_t)min(first, max_chunks);
-            for (int64_t c = 0; c < cnt && first + c < max_chunks; ++c) {
-                Chunk ch;
-                ch.start = lo + c * chunk;
-                ch.len = (int32_t)min(chunk, hi - ch.start);
-                ch.group = (int32_t)g;
-                table[first + c] = ch;
-            }
-        }
-        __syncthreads();
-        if (tid == (int)blockDim.x - 1) base_s = base + scan[tid];
-        __syncthreads();
+// Generation of a launch: distinct for every call of the process (48 bits,
+// never 0), starting from a value taken from the clock so that a workspace
+// left by another process is unlikely to hold a matching stamp.
+unsigned long long next_generation() {
+    static std::atomic<unsigned long long> g{
+        ((unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull) >>
+        16};
+    for (;;) {
+        const unsigned long long v = (g.fetch_add(1, std::memory_order_relaxed) + 1) & kGenMask;
+        if (v != 0) return v;
     }
-    if (tid == 0) {
-        const int64_t n = min(base_s, max_chunks);
-        kfirst[G] = (int32_t)n;
-        *n_chunks_out = (int32_t)n;
-        // only overlapping (decreasing) offsets hold more chunks than the bound; the chunks
-        // past it are dropped and the call reports it
-        if (base_s > max_chunks) atomicExch(status, (int)LH_ERR_INVALID_ARG);
-    }
-}
-
-// H[g][j][e] = fp32(H[g][j][e] + sum_{k in chunks of g} partial[k][j][e]) in FP64, chunk order.
-// One block per group and `cols` (8) block columns: each thread keeps 8 independent
-// sums, so the loads of a chunk are in flight together (many groups, few chunks each).
-__global__ void __launch_bounds__(256) hessian_reduce_kernel(const float* __restrict__ partial,
-                                                             const int32_t* __restrict__ kfirst, int64_t J,
-                                                             int64_t n_chunks_plain, int cols,
-                                                             float* __restrict__ H) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials of the kernel before
-    const int64_t j0 = (int64_t)blockIdx.x * cols;
-    const int64_t g = blockIdx.y;
-    const int e = threadIdx.x;
-    int64_t k0, k1;
-    if (kfirst) { k0 = kfirst[g]; k1 = kfirst[g + 1]; }
-    else { k0 = 0; k1 = n_chunks_plain; }
-    if (k1 <= k0) return;
-    const int nj = (int)min((int64_t)cols, J - j0);
-    float* h = H + ((size_t)g * J + j0) * 256 + e;
-    double hs[8], acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        hs[i] = i < nj ? (double)h[i * 256] : 0.0;
-        acc[i] = 0.0;
-    }
-    for (int64_t k = k0; k < k1; ++k) {
-        const float* src = partial + ((size_t)k * J + j0) * 256 + e;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i < nj) acc[i] += (double)src[i * 256];
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (i < nj) h[i * 256] = (float)(hs[i] + acc[i]);
-}
-
-
-// The same with one block column per block (one group: enough blocks to fill the GPU).
-__global__ void __launch_bounds__(256) hessian_reduce1_kernel(const float* __restrict__ partial,
-                                                              const int32_t* __restrict__ kfirst, int64_t J,
-                                                              int64_t n_chunks_plain, float* __restrict__ H) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials of the kernel before
-    const int64_t j = blockIdx.x;
-    const int64_t g = blockIdx.y;
-    const int e = threadIdx.x;
-    int64_t k0, k1;
-    if (kfirst) { k0 = kfirst[g]; k1 = kfirst[g + 1]; }
-    else { k0 = 0; k1 = n_chunks_plain; }
-    if (k1 <= k0) return;
-    double s = 0.0;
-    for (int64_t k = k0; k < k1; ++k) s += (double)partial[((size_t)k * J + j) * 256 + e];
-    float* h = H + ((size_t)g * J + j) * 256 + e;
-    *h = (float)((double)*h + s);
 }
 
 // Argument checks shared by the Hessian entry points (host side, before any launch).
@@ -490,28 +578,34 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
+
 }  // namespace
 }  // namespace lh
 
 extern "C" size_t lh_hessian_workspace_bytes(int64_t n_tokens_total, int64_t c_in, int64_t n_groups) {
+    using namespace lh;
     if (n_tokens_total < 0 || c_in <= 0 || n_groups < 1) return 0;
-    return lh::make_plan(n_tokens_total, c_in, n_groups).ws.total;
+    // sized for the largest grid the launch uses on any GPU (it uses fewer CTAs on one with
+    // under 160 SMs, and then fewer bands and parts)
+    return ws_layout(make_grid(n_tokens_total, c_in, kMaxCtas)).total;
 }
 
 extern "C" lh_status lh_workspace_status(const void* workspace, void* stream) {
     using namespace lh;
     clear_error();
     if (!workspace) return fail(LH_ERR_INVALID_ARG, "null workspace");
-    int err = 0;
+    unsigned long long w[2] = {0, 0};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    lh_status s = cuda_status(cudaMemcpyAsync(&err, workspace, sizeof(int), cudaMemcpyDeviceToHost, st),
+    lh_status s = cuda_status(cudaMemcpyAsync(w, workspace, sizeof(w), cudaMemcpyDeviceToHost, st),
                               "read workspace status");
     if (s != LH_OK) return s;
     s = cuda_status(cudaStreamSynchronize(st), "synchronise");
     if (s != LH_OK) return s;
+    if ((w[0] >> 16) != (w[1] & kGenMask)) return LH_OK;  // no error recorded by the last launch
+    const int err = (int)(w[0] & 0xFFFFull);
     if (err == LH_ERR_TIMEOUT) return fail(LH_ERR_TIMEOUT, "a bounded wait in the Hessian kernel expired");
-    if (err != 0)
-        return fail((lh_status)err, "the group offsets overlap: their ranges hold more tokens than n_tokens_total");
+    if (err == LH_ERR_INVALID_ARG) return fail(LH_ERR_INVALID_ARG, "the group offsets decrease (overlapping ranges)");
+    if (err != 0) return fail((lh_status)err, "the Hessian kernel recorded an error");
     return LH_OK;
 }
 
@@ -524,9 +618,8 @@ extern "C" lh_status lh_debug_wait_timeout(void* workspace, size_t workspace_byt
         return fail(LH_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
     if (timeout_us < 1 || timeout_us > 1000000) return fail(LH_ERR_INVALID_ARG, "timeout_us must be in [1, 1e6]");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    lh_status s = cuda_status(cudaMemsetAsync(workspace, 0, kHeaderBytes, st), "clear workspace header");
-    if (s != LH_OK) return s;
-    wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<int*>(workspace), (uint64_t)timeout_us * 1000ull, arrive);
+    wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<unsigned long long*>(workspace), next_generation(),
+                                          (uint64_t)timeout_us * 1000ull, arrive);
     return cuda_status(cudaGetLastError(), "wait_timeout_kernel launch");
 }
 
@@ -538,9 +631,9 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     lh_status s = validate_hessian_args(X, x_dtype, n_tokens_total, c_in, ld_x, offsets, n_groups, H);
     if (s != LH_OK) return s;
     if (n_tokens_total == 0 || c_in == 0) return LH_OK;
-    const Plan plan = make_plan(n_tokens_total, c_in, n_groups);
-    if (!workspace || workspace_bytes < plan.ws.total)
-        return fail(LH_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.ws.total,
+    const WsLayout wl = ws_layout(make_grid(n_tokens_total, c_in, kMaxCtas));  // what the workspace is sized for
+    if (!workspace || workspace_bytes < wl.total)
+        return fail(LH_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", wl.total,
                     workspace ? workspace_bytes : (size_t)0);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(LH_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
@@ -549,89 +642,64 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     auto encode = get_encode_fn();
     if (!encode) return fail(LH_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
 
-    CUtensorMap tmap;
+    CUtensorMap tmap, tmap16;
     const cuuint64_t dims[2] = {(cuuint64_t)c_in, (cuuint64_t)n_tokens_total};
     const cuuint64_t strides[1] = {(cuuint64_t)(ld_x * 2)};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kStageTok};
     const cuuint32_t estr[2] = {1, 1};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kStageTok};
+    const cuuint32_t box16[2] = {64, (cuuint32_t)kSmallBox};
     CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr == CUDA_SUCCESS)
+        cr = encode(&tmap16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(X), dims, strides, box16, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS) return fail(LH_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)cr);
 
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t cap = 2 * (int64_t)sms < kMaxCtas ? 2 * (int64_t)sms : kMaxCtas;  // two CTAs per SM
+    const Grid gr = make_grid(n_tokens_total, c_in, cap);  // no more bands or slabs than sized for
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    s = cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, st), "clear workspace header");
-    if (s != LH_OK) return s;
-
-    const int64_t J = c_in / 16;
     KParams kp;
-    kp.n_tok = n_tokens_total;
-    kp.J = J;
-    kp.n_slabs = plan.n_slabs;
-    kp.chunk = plan.chunk;
-    kp.n_items_max = plan.max_chunks * plan.n_slabs;
-    kp.grouped = offsets != nullptr;
-    kp.table = reinterpret_cast<const Chunk*>(ws + plan.ws.table_off);
-    kp.n_chunks_dev = reinterpret_cast<const int32_t*>(ws + 4);
-    kp.partial = reinterpret_cast<float*>(ws + plan.ws.partial_off);
-    kp.err = reinterpret_cast<int*>(ws);
-    int32_t* kfirst = reinterpret_cast<int32_t*>(ws + plan.ws.kfirst_off);
-
-    if (offsets) {
-        chunk_table_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, n_tokens_total, plan.chunk, plan.max_chunks,
-                                               reinterpret_cast<Chunk*>(ws + plan.ws.table_off), kfirst,
-                                               reinterpret_cast<int32_t*>(ws + 4), reinterpret_cast<int*>(ws));
-        s = cuda_status(cudaGetLastError(), "chunk_table_kernel launch");
-        if (s != LH_OK) return s;
-    }
+    kp.N = n_tokens_total;
+    kp.J = c_in / 16;
+    kp.G = offsets ? n_groups : 1;
+    kp.slabs = gr.slabs;
+    kp.sgroups = gr.sgroups;
+    kp.bands = gr.bands;
+    kp.off = offsets;
+    kp.H = H;
+    kp.hdr = reinterpret_cast<unsigned long long*>(ws);
+    kp.parts = reinterpret_cast<float*>(ws + wl.part_off);
+    kp.gen = next_generation();
 
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
-    const size_t smem_bytes = (size_t)kStages * kStageBytes + 1024 + 256;
+    const size_t smem_bytes = (size_t)kStages * kStageBytes + 1024 + sizeof(Smem);
     std::call_once(attr_once, [&] {
         attr_err = cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
     });
     if (attr_err != cudaSuccess) return cuda_status(attr_err, "set shared memory size");
-    int64_t grid = kp.n_items_max < 2 * sms ? kp.n_items_max : 2 * sms;  // two CTAs per SM
-    {
-        // programmatic launch: the set-up of its blocks overlaps the end of the kernel before
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)grid);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem_bytes;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        s = cuda_status(cudaLaunchKernelEx(&cfg, hessian_tc_kernel, tmap, kp), "hessian_tc_kernel launch");
-    }
-    if (s != LH_OK) return s;
-
-    const int64_t plain_chunks = (n_tokens_total + plan.chunk - 1) / plan.chunk;
-    {
-        // launched as a programmatic dependent of the main kernel: its blocks start while
-        // that kernel drains and wait (griddepcontrol.wait) for its partial sums
-        const int cols = (n_groups * ((J + 7) / 8) >= 4 * (int64_t)sms) ? 8 : 1;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)((J + cols - 1) / cols), (unsigned)n_groups);
-        cfg.blockDim = dim3(256);
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const float* part = kp.partial;
-        const int32_t* kf = offsets ? kfirst : nullptr;
-        s = cols == 1 ? cuda_status(cudaLaunchKernelEx(&cfg, hessian_reduce1_kernel, part, kf, J, plain_chunks, H),
-                                    "hessian_reduce1_kernel launch")
-                      : cuda_status(cudaLaunchKernelEx(&cfg, hessian_reduce_kernel, part, kf, J, plain_chunks, cols, H),
-                        "hessian_reduce_kernel launch");
-    }
-    return s;
+    // programmatic launch: the set-up of its CTAs overlaps the end of the kernel before
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)gr.ctas());
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    s = cuda_status(cudaLaunchKernelEx(&cfg, hessian_tc_kernel, tmap, tmap16, kp), "hessian_tc_kernel launch");
+    if (s != LH_OK || gr.bands == 1) return s;
+    // the parts of segments that several bands share (a programmatic dependent as well)
+    cudaLaunchConfig_t cfg2 = cfg;
+    cfg2.gridDim = dim3((unsigned)gr.slabs, (unsigned)(gr.bands - 1));
+    cfg2.blockDim = dim3(kPartsThreads);
+    cfg2.dynamicSmemBytes = 0;
+    return cuda_status(cudaLaunchKernelEx(&cfg2, hessian_parts_kernel, kp), "hessian_parts_kernel launch");
 }
 
 // ---------------------------------------------------------------------------
@@ -650,19 +718,23 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
 // address; its device address is looked up once per device with
 // cudaGetSymbolAddress on the first call made with that device current, and
 // that lookup is the only set-up. Make the first call on each device before
-// any stream capture. All calls share the one array: the header words that
-// must start at zero are cleared by every call, and calls whose kernels
-// overlap on the GPU (different streams, or different host threads) race on
-// the array and must be serialised by the caller.
+// any stream capture. All calls share the one array: nothing in it needs
+// clearing between calls (its parts are rewritten before they are read and its status word carries each call's
+// generation), and calls whose kernels overlap on the GPU (different streams,
+// or different host threads) race on the array and must be serialised by the
+// caller.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;  // 16 MiB
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
 }  // namespace
 
 static __device__ __align__(256) unsigned char lh_noalloc_scratch[kNoAllocScratchBytes];
+// the largest workspace (parts of kMaxCtas (band, slab) pairs) fits: no call is turned away
+static_assert(lh::ws_layout(lh::Grid{1, 1, lh::kMaxCtas}).total <= kNoAllocScratchBytes,
+              "scratch holds the largest workspace");
 
 // Device address of the scratch array for the current device, looked up on
 // first use with that device current (the only set-up the entry point needs).
@@ -693,10 +765,10 @@ extern "C" lh_status lh_accumulate_hessian_noalloc(const void* X, lh_dtype x_dty
     if (s != LH_OK) return s;
     if (n_tokens_total == 0 || c_in == 0) return LH_OK;
     const size_t need = lh_hessian_workspace_bytes(n_tokens_total, c_in, n_groups);
-    if (need > kNoAllocScratchBytes)
+    if (need > kNoAllocScratchBytes)  // cannot happen (see the static_assert); kept as a guard
         return fail(LH_ERR_WORKSPACE,
                     "this Hessian needs %zu bytes of scratch but the allocation-free entry point has %zu "
-                    "(16 MiB); call lh_accumulate_hessian with a caller-provided workspace instead",
+                    "(8 MiB); call lh_accumulate_hessian with a caller-provided workspace instead",
                     need, kNoAllocScratchBytes);
     void* scratch = nullptr;
     s = noalloc_scratch(&scratch);

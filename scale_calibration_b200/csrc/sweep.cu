@@ -13,8 +13,8 @@
 //    takes a tile of 1024 rows of one block column (the last wave of tiles is
 //    cut into 512- and 256-row pieces so the launch drains quickly), stages H_j once in
 //    shared memory (read by broadcast), sorts the tile's rows by the largest
-//    |w| over the heavy channels, and hands out 32-row chunks of the sorted
-//    order to its four warps.
+//    |w| over the heavy channels (to 1/16 of an octave), and hands out 32-row
+//    chunks of the sorted order to its four warps.
 //  * Candidate scales come in 8 mantissa classes (1 + f/8) * 2^x. Within a
 //    class consecutive codes double the scale exactly, so fp32(w / s_c) is
 //    fp32(w / s_c0) scaled by a power of two: 16 correctly rounded quotients
@@ -80,18 +80,19 @@ __device__ __forceinline__ int class_code(int f, int x) {
     return x >= -6 ? 8 * (x + 7) + f : (8 + f) >> (-6 - x);
 }
 
-// Correctly rounded FP32 quotient a / b for positive normal b, from y = RN(1/b)
-// (correctly rounded reciprocal): q = RN(a y) is within one ulp of a/b, the
-// remainder a - b q is exact with one FMA, and RN(q + r y) is RN(a/b)
-// (P. Markstein, "Computation of elementary functions on the IBM RISC
-// System/6000 processor", IBM J. Res. Dev. 34(1), 1990, Theorem 1; see also
-// Muller et al., Handbook of Floating-Point Arithmetic, ch. 4). Valid while
-// the remainder a - b q cannot underflow, i.e. for a >= 2^-100 (or a = 0)
-// and a normal b; blocks with a smaller non-zero |w| use IEEE division.
-__device__ __forceinline__ float div_by_recip(float a, float b, float y) {
-    const float q = __fmul_rn(a, y);
-    const float r = __fmaf_rn(-q, b, a);
-    return __fmaf_rn(r, y, q);
+// Correctly rounded FP32 quotients a / b for positive normal b, two lanes at
+// once, from y = RN(1/b) (correctly rounded reciprocal): q = RN(a y) is within
+// one ulp of a/b, the remainder a - b q is exact with one FMA, and RN(q + r y)
+// is RN(a/b) (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990, Theorem 1; see
+// also Muller et al., Handbook of Floating-Point Arithmetic, ch. 4). Valid
+// while the remainder a - b q cannot underflow, i.e. for a >= 2^-100 (or a = 0)
+// and a normal b; blocks with a smaller non-zero |w| use IEEE division. The
+// packed FP32 operations round each lane exactly as the scalar ones; nb = -b.
+__device__ __forceinline__ float2 div_by_recip2(float2 a, float2 nb, float2 y) {
+    const float2 q = __fmul2_rn(a, y);
+    const float2 r = __ffma2_rn(q, nb, a);
+    return __ffma2_rn(r, y, q);
 }
 
 // IEEE quotients w_i / s0 for blocks holding a tiny non-zero weight (rare;
@@ -206,6 +207,7 @@ struct SweepShared {
     float mu;               // mu <= lambda_min(D^-1/2 H D^-1/2), D = diag(H); 0 disables pruning
     float nu;               // nu >= lambda_max(|D^-1/2 H D^-1/2|) (largest absolute row sum)
     int next_chunk;         // next 32-row chunk of the sorted order to hand to a warp
+    unsigned kmax;          // largest sort key of the tile
     // the CTA's unit, read back in the row loop rather than kept in registers
     unsigned long long wcol;  // address of W[m][tile0][16 j]
     long long ocol;           // index of output (m, tile0, j)
@@ -397,10 +399,14 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
     // the optimum lies; each class's walk starts at its max-scaling step. After
     // sorting, the 32 rows of a warp mostly agree on where to start, what to skip
     // and when to stop.
-    // counting sort of the tile's rows by a 9-bit key (exponent and first
-    // mantissa bit of that largest |w|; rows past c_out last)
+    // counting sort of the tile's rows by a 9-bit key: the octaves below the tile's
+    // largest key (up to 30) and the first four mantissa bits of that largest |w|, so
+    // rows within 1/16 of each other share a bucket; rows past c_out last
     for (int i = tid; i < kSortBuckets; i += kThreads) sm.hist[i] = 0;
-    if (tid == 0) sm.next_chunk = 0;
+    if (tid == 0) {
+        sm.next_chunk = 0;
+        sm.kmax = 0u;
+    }
     __syncthreads();
     uint32_t kb[kRowsPerThread];
 #pragma unroll
@@ -418,10 +424,26 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 mh = ((heavy >> i) & 1u) ? fmaxf(mh, fabsf(wk[i])) : mh;
             }
             key = __float_as_uint(mh > 0.0f ? mh : mx);
+            atomicMax(&sm.kmax, key);  // non-negative floats order like their bits
         }
-        kb[q] = (key == 0xFFFFFFFFu) ? (uint32_t)(kSortBuckets - 1) : min(key >> 22, (uint32_t)(kSortBuckets - 2));
+        kb[q] = key;
         sm.key[p] = ((unsigned long long)key << 32) | (unsigned)p;
-        atomicAdd(&sm.hist[kb[q]], 1u);
+    }
+    __syncthreads();
+    // buckets, largest keys first
+    {
+        const uint32_t emax = sm.kmax >> 23;
+#pragma unroll
+        for (int q = 0; q < kRowsPerThread; ++q) {
+            const uint32_t key = kb[q];
+            if (key == 0xFFFFFFFFu) {
+                kb[q] = kSortBuckets - 1;
+            } else {
+                const uint32_t d = min(emax - min(key >> 23, emax), 30u);
+                kb[q] = d * 16u + (15u - ((key >> 19) & 15u));
+            }
+            atomicAdd(&sm.hist[kb[q]], 1u);
+        }
     }
     __syncthreads();
     if (tid < 32) {  // exclusive scan of the histogram by one warp
@@ -587,9 +609,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     quotients_ieee(w, s0, u);
                 } else {
                     const float rs0 = __frcp_rn(s0);
+                    const float2 ns02 = make_float2(-s0, -s0), rs02 = make_float2(rs0, rs0);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p)
-                        u[p] = make_float2(div_by_recip(w[2 * p], s0, rs0), div_by_recip(w[2 * p + 1], s0, rs0));
+                    for (int p = 0; p < 8; ++p) u[p] = div_by_recip2(w2[p], ns02, rs02);
                 }
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {

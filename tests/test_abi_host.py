@@ -95,8 +95,8 @@ def test_hessian_rejects_bad_arguments():
 
 
 def test_hessian_noalloc_checks_arguments_like_the_workspace_entry():
-    # the allocation-free entry point returns the same argument errors, before its size limit
-    # and before touching any device (no GPU here)
+    # the allocation-free entry point returns the same argument errors, before touching any
+    # device (no GPU here)
     lh = _lh()
     ok = dict(X=FAKE, x_dtype=lh.LH_BF16, n_tokens_total=300, c_in=64, ld_x=64, offsets=None, n_groups=1, H=FAKE,
               stream=0, check=False)
@@ -104,18 +104,27 @@ def test_hessian_noalloc_checks_arguments_like_the_workspace_entry():
         (dict(x_dtype=lh.LH_F32), 2), (dict(X=0), 1), (dict(H=0), 1), (dict(n_groups=2), 1),
         (dict(c_in=40, ld_x=40), 2), (dict(ld_x=60), 1), (dict(ld_x=68), 3), (dict(X=FAKE + 8), 3),
         (dict(n_tokens_total=-1), 1), (dict(n_groups=0), 1),
-        # far beyond the 16 MiB scratch, but the argument error comes first
         (dict(n_tokens_total=1 << 24, c_in=40008, ld_x=40008), 2),
         (dict(n_tokens_total=1 << 24, c_in=32768, ld_x=32768, X=0), 1),
     ]
     for over, want in cases:
         a = dict(ok, **over)
         assert lh.lh_accumulate_hessian_noalloc(**a) == want, over
-    # valid arguments beyond the scratch: LH_ERR_WORKSPACE, still before any device call
-    a = dict(ok, n_tokens_total=1 << 24, c_in=32768, ld_x=32768)
-    assert lh.lh_accumulate_hessian_noalloc(**a) == 4
-    assert "16 MiB" in lh.lh_last_error_message()
     assert lh.lh_accumulate_hessian_noalloc(**dict(ok, n_tokens_total=0)) == 0
+
+
+def test_hessian_workspace_is_bounded_and_fits_the_noalloc_scratch():
+    # the Hessian kernel runs at most 320 CTAs (token bands x slabs) and the workspace holds at
+    # most two parts per CTA: it stops growing with the tokens, never depends on the groups,
+    # and the largest one fits the 8 MiB array of the allocation-free entry point
+    lh = _lh()
+    sizes = [lh.lh_hessian_workspace_bytes(n, c, g) for n in (1, 255, 4096, 1 << 20, (1 << 31) - 1)
+             for c in (16, 2048, 4096, 17408, 40960, (1 << 31) - 16) for g in (1, 64, 65535)]
+    assert 0 < max(sizes) <= (8 << 20)
+    assert lh.lh_hessian_workspace_bytes(1 << 20, 4096, 1) == lh.lh_hessian_workspace_bytes(4096, 4096, 64)
+    assert lh.lh_hessian_workspace_bytes(256, 128, 1) < lh.lh_hessian_workspace_bytes(2048, 128, 1)
+    # a layer wider than the grid runs as one band: no parts at all
+    assert lh.lh_hessian_workspace_bytes(4096, 128 * 400, 1) == 256
 
 
 def test_hessian_zero_tokens_is_noop():
@@ -123,13 +132,13 @@ def test_hessian_zero_tokens_is_noop():
     assert lh.lh_accumulate_hessian(FAKE, lh.LH_BF16, 0, 64, 64, None, 1, FAKE, 0, 0, 0, check=False) == 0
 
 
-def test_workspace_size_grows_with_tokens_and_groups():
+def test_workspace_size_grows_with_tokens_then_stays_bounded():
     lh = _lh()
-    a = lh.lh_hessian_workspace_bytes(2048, 4096, 1)
-    b = lh.lh_hessian_workspace_bytes(16384, 4096, 1)
+    a = lh.lh_hessian_workspace_bytes(256, 128, 1)
+    b = lh.lh_hessian_workspace_bytes(2048, 128, 1)
     c = lh.lh_hessian_workspace_bytes(2048, 4096, 64)
-    J = 4096 // 16
-    assert a >= 256 + J * 1024 and b >= a and c > a
+    d = lh.lh_hessian_workspace_bytes(16384, 4096, 1)
+    assert 0 < a < b <= c == d
     assert lh.lh_hessian_workspace_bytes(100, 0, 1) == 0
 
 

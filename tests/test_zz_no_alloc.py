@@ -13,7 +13,6 @@ import pytest
 import torch
 
 import synth
-from scale_calibration_b200._binding import LH_ERR_WORKSPACE
 from tests import gpu_util as gu
 
 pytestmark = pytest.mark.gpu
@@ -49,9 +48,9 @@ def test_noalloc_matches_workspace_entry_on_consecutive_calls(cuda_ok):
 
 
 def test_noalloc_reports_kernel_side_errors_through_its_status(cuda_ok):
-    # two groups over the same 1000 tokens hold more chunks than the scratch's chunk table
-    # allows: the kernels stay in bounds and record the error in the scratch header, which
-    # lh_noalloc_status reads; the next valid call clears it
+    # decreasing offsets (two groups over the same 1000 tokens): the kernel stays in bounds
+    # and records the error in the scratch's status word, which lh_noalloc_status reads; the
+    # next valid call leaves no error
     import scale_calibration_b200 as lh
     layer = synth.make_layer(8, 128, 1000, seed=32)
     _, X, _ = gu.to_device(layer)
@@ -63,15 +62,3 @@ def test_noalloc_reports_kernel_side_errors_through_its_status(cuda_ok):
     H1 = torch.zeros(1, 8, 16, 16, device="cuda")
     lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, 1000, 128, 128, None, 1, H1)
     assert lh.lh_noalloc_status() == 0
-
-
-def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
-    import scale_calibration_b200 as lh
-    n_tok, c_in, n_groups = 4096, 32768, 64   # one partial slot per (slab, group): far more than 16 MiB
-    assert lh.lh_hessian_workspace_bytes(n_tok, c_in, n_groups) > (16 << 20)
-    H = torch.zeros(1, dtype=torch.float32, device="cuda")
-    X = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
-    off = torch.zeros(n_groups + 1, dtype=torch.int64, device="cuda")
-    s = lh.lh_accumulate_hessian_noalloc(X, lh.LH_BF16, n_tok, c_in, c_in, off, n_groups, H, check=False)
-    assert s == LH_ERR_WORKSPACE
-    assert "16 MiB" in lh.lh_last_error_message()
