@@ -44,7 +44,7 @@ UNIT = "blocks/s"
 SWEEP_FLOP_PER_BLOCK = 126 * 152 * 2   # 16 dw FMA + 136 symmetric-form FMA per candidate
 FP32_LANES_PER_SM = 128
 # kernels of ours launched per call (counted in the timed region's gpu_launches)
-LAUNCHES = dict(absmax=2, hessian_plain=1, hessian_grouped=1, sweep_ws=2, fake_quant=1)
+LAUNCHES = dict(absmax=2, hessian_plain=2, hessian_grouped=2, sweep_ws=2, fake_quant=1)  # Hessian: main + parts kernel
 
 
 def profiled_traffic(kernel_src: str, summary: str):
@@ -272,6 +272,54 @@ def fma_probe(lh, torch, dev, stream) -> dict:
             ts.append(e0.elapsed_time(e1) / 1e3)
         res[name] = lh.lh_probe_fma_flop(blocks, iters) / min(ts) / 1e12
     return res
+
+
+def sweep_work(lh, torch, dev, s, W, n_mats, c_out, c_in, ld, amax, H, codes, t_sweep_ms, fp32_peak):
+    """What the sweep executes, from its measurement build (liblh_counters.so, the
+    same sources with work counters compiled in): one extra untimed call on the
+    same inputs, whose codes must equal the timed library's. The executed FP32 work
+    counts 272 flop per full form (136 FMA) and 64 per quantised candidate (16 FMA
+    for dw, 16 for the diagonal bound), per block; its rate uses the timed sweep."""
+    import ctypes
+    path = os.path.join(ROOT, "scale_calibration_b200", "liblh_counters.so")
+    if not os.path.exists(path):
+        return None
+    lib = ctypes.CDLL(path)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    lib.lh_sweep_scales_ws.argtypes = [P, I32, I64, I64, I64, I64, P, P, P, P, P, SZ, P]
+    lib.lh_sweep_scales_ws.restype = I32
+    lib.lh_sweep_workspace_bytes.argtypes = [I64, I64]
+    lib.lh_sweep_workspace_bytes.restype = SZ
+    lib.lh_debug_sweep_counts.argtypes = [P, I32]
+    lib.lh_debug_sweep_counts.restype = I32
+    wsb = lib.lh_sweep_workspace_bytes(n_mats, c_in)
+    wsp = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    c2 = torch.empty_like(codes)
+    a2 = torch.empty(codes.shape, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+    if lib.lh_debug_sweep_counts(None, 1) != 0:
+        return None
+    dt = lh.LH_BF16 if W.dtype == torch.bfloat16 else lh.LH_F32
+    st = lib.lh_sweep_scales_ws(W.data_ptr(), dt, n_mats, c_out, c_in, ld, amax.data_ptr(), H.data_ptr(),
+                                a2.data_ptr(), c2.data_ptr(), wsp.data_ptr(), wsb, s)
+    torch.cuda.synchronize(dev)
+    cnt = (ctypes.c_uint64 * 8)()
+    if st != 0 or lib.lh_debug_sweep_counts(cnt, 0) != 0:
+        return None
+    chunks, blocks, cand, forms, need, below, resweep, classes = (int(x) for x in cnt)
+    if blocks == 0:
+        return None
+    fpb = 32.0 * forms / blocks
+    qpb = 32.0 * cand / blocks
+    flop = 272.0 * fpb + 64.0 * qpb
+    tf = flop * blocks / (t_sweep_ms / 1e3) / 1e12
+    return dict(forms_per_block=fpb, lane_needed_forms_per_block=need / blocks,
+                candidates_quantised_per_block=qpb, class_bound_tests_per_block=32.0 * below / blocks,
+                fp64_resweeps_per_1000_blocks=1000.0 * resweep / blocks, flop_per_block=flop,
+                achieved=tf, unit="TFLOP/s", frac=tf / fp32_peak, same_codes=bool(torch.equal(codes, c2)),
+                note="measurement build (liblh_counters.so): forms and candidates are counted per 32-lane warp, "
+                     "so every lane pays for a form any lane needs; flop = 272 per form + 64 per quantised "
+                     "candidate, over the timed sweep")
 
 
 def make_share(layer, rank: int, ws: int) -> dict:
@@ -570,6 +618,10 @@ def run_ours(args):
                     fma_probe=probe, flop_per_block=SWEEP_FLOP_PER_BLOCK, blocks_per_launch=int(s_blocks))
     if clocks.get("sm_mhz"):
         roofline["frac_at_measured_clock"] = sweep_tflops / (fp32_peak * clocks["sm_mhz"] / peaks["sm_max_mhz"])
+    if s_blocks:
+        ex = sweep_work(lh, torch, dev, s, W, s_mats, s_out, s_cin, ld, amax, sweep_h(H), codes, t_sweep, fp32_peak)
+        if ex:
+            roofline["executed"] = ex
     hessian = dict(tokens_per_s=n_loc / (t_hess / 1e3) if t_hess > 0 else None, bound="hbm",
                    achieved=hess_gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=hess_gbs / peaks["hbm_gbs"],
                    bytes_per_launch=hess_bytes, peak_source=peaks["source"],

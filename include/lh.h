@@ -141,6 +141,16 @@ LH_API lh_status lh_debug_wait_timeout(void* workspace, size_t workspace_bytes, 
 LH_API int64_t lh_probe_fma_flop(int64_t blocks, int64_t iters);
 LH_API lh_status lh_probe_fma(int packed, int64_t blocks, int64_t iters, float* out, void* stream);
 
+/* Diagnostics; the pages have no counterpart. Work counters of the sweep,
+ * summed over the launches since the last clear: out[8] = {warp chunks of 32
+ * rows, blocks, candidates quantised per warp, full quadratic forms evaluated
+ * per warp, forms some lane needed (lane count), class-wide bound tests, blocks
+ * re-swept in FP64, mantissa classes walked per warp}. clear != 0 zeroes them
+ * (out unused). Only a library built with -DLH_SWEEP_COUNTERS=1 (the
+ * measurement build, liblh_counters.so) counts; the library itself returns
+ * LH_ERR_UNSUPPORTED. Synchronous. */
+LH_API lh_status lh_debug_sweep_counts(uint64_t* out, int clear);
+
 /* ------------------------------------------------------------------------
  * Allocation-free variant of lh_accumulate_hessian. The pages have no
  * counterpart: this is a library convenience for callers that cannot

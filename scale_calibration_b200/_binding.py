@@ -20,7 +20,7 @@ EXPORTS = [
     "lh_status_string", "lh_last_error_message", "lh_absmax", "lh_hessian_workspace_bytes",
     "lh_accumulate_hessian", "lh_workspace_status", "lh_sweep_scales", "lh_fake_quant",
     "lh_accumulate_hessian_noalloc", "lh_noalloc_status", "lh_debug_wait_timeout", "lh_quantize_nvfp4", "lh_baseline_scales",
-    "lh_search_amax", "lh_sweep_workspace_bytes", "lh_sweep_scales_ws", "lh_probe_fma", "lh_probe_fma_flop",
+    "lh_search_amax", "lh_sweep_workspace_bytes", "lh_sweep_scales_ws", "lh_probe_fma", "lh_probe_fma_flop", "lh_debug_sweep_counts",
 ]
 LH_SCALE_MAX, LH_SCALE_FOUR_OVER_SIX, LH_SCALE_MSE = range(3)
 
@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "lh_search_amax": (I32, [P, I32, I64, I64, I64, I64, P, P, ctypes.c_double, ctypes.c_double, I64, P, P, P]),
         "lh_probe_fma_flop": (I64, [I64, I64]),
         "lh_probe_fma": (I32, [I32, I64, I64, P, P]),
+        "lh_debug_sweep_counts": (I32, [P, I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

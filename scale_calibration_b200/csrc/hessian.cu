@@ -696,7 +696,8 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     if (s != LH_OK || gr.bands == 1) return s;
     // the parts of segments that several bands share (a programmatic dependent as well)
     cudaLaunchConfig_t cfg2 = cfg;
-    cfg2.gridDim = dim3((unsigned)gr.slabs, (unsigned)(gr.bands - 1));
+    // one group (no offsets): only boundary 1 of each slab starts a segment, so one CTA per slab
+    cfg2.gridDim = dim3((unsigned)gr.slabs, offsets ? (unsigned)(gr.bands - 1) : 1u);
     cfg2.blockDim = dim3(kPartsThreads);
     cfg2.dynamicSmemBytes = 0;
     return cuda_status(cudaLaunchKernelEx(&cfg2, hessian_parts_kernel, kp), "hessian_parts_kernel launch");

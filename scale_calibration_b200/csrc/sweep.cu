@@ -36,6 +36,18 @@
 #include "common.cuh"
 #include "quant.cuh"
 
+// Measurement build only (-DLH_SWEEP_COUNTERS=1): the work the walk does, summed
+// over a launch; lh_debug_sweep_counts reads and clears it. Off in the library.
+#ifndef LH_SWEEP_COUNTERS
+#define LH_SWEEP_COUNTERS 0
+#endif
+#if LH_SWEEP_COUNTERS
+// [0] warp chunks, [1] blocks, [2] candidates quantised (per warp), [3] full forms (per
+// warp), [4] forms a lane needed (its bound did not exclude the candidate), [5] class-wide
+// bound tests, [6] blocks re-swept in FP64, [7] classes walked (per warp)
+__device__ unsigned long long lh_sweep_counts[8];
+#endif
+
 #ifndef LH_SWEEP_UREGS
 #define LH_SWEEP_UREGS false  // form coefficients read from shared memory (more warps per SM)
 #endif
@@ -541,6 +553,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
             if constexpr (kMask) return (sm.allow[code >> 5][t] >> (code & 31)) & 1u;
             else return true;
         };
+#if LH_SWEEP_COUNTERS
+        unsigned cnt_cand = 0, cnt_form = 0, cnt_need = 0, cnt_below = 0, cnt_class = 0;
+#endif
         float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
         int best_fk = -1;  // 32 f + k of the best candidate (class f, step k); the code is formed at the end
         bool flag = !fast;
@@ -596,6 +611,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 
 #pragma unroll 1
             for (int f = 0; f < 8; ++f) {
+#if LH_SWEEP_COUNTERS
+                ++cnt_class;
+#endif
                 const int tz = (f == 0) ? 3 : (f == 4) ? 2 : (f == 2 || f == 6) ? 1 : 0;
                 const int x0 = -6 - tz;                  // smallest exponent of the class
                 const int n = (f == 7 ? 7 : 8) - x0 + 1;  // codes in the class
@@ -623,6 +641,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 // One candidate; returns true (upward walk only) when every lane proves that no
                 // later candidate of the upward walk can beat the incumbent.
                 auto candidate = [&](int k, bool up) -> bool {
+#if LH_SWEEP_COUNTERS
+                    ++cnt_cand;
+#endif
                     const float lim = __int_as_float(((129 + k) << 23) | 0x400000);  // 6 * 2^k
                     const unsigned mlo = ((unsigned)(127 + k) << 23) + 0x0B400000u;
                     float E;
@@ -738,6 +759,10 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                             }
                         } else {
                             E = form(dw);
+#if LH_SWEEP_COUNTERS
+                            ++cnt_form;
+                            cnt_need += __popc(__ballot_sync(0xFFFFFFFFu, !out && active));
+#endif
                         }
                     }
                     if constexpr (kMask) {
@@ -757,6 +782,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 // when, for every lane, that bound already exceeds the incumbent's error.
                 auto below_excluded = [&](int k1) -> bool {
                     if (!rel) return false;
+#if LH_SWEEP_COUNTERS
+                    ++cnt_below;
+#endif
                     const float thr = best_e * up_fac;
                     const float nc3 = -__int_as_float(((128 + k1) << 23) | 0x400000);  // -3 * 2^k1
                     float2 acc = make_float2(0.0f, 0.0f), acc2 = make_float2(0.0f, 0.0f);
@@ -811,6 +839,21 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 
         // FP64 re-sweep of flagged blocks, one block at a time across the warp.
         unsigned pending = __ballot_sync(0xFFFFFFFFu, flag && active);
+#if LH_SWEEP_COUNTERS
+        {
+            const unsigned act = __ballot_sync(0xFFFFFFFFu, active);
+            if (lane == 0) {
+                atomicAdd(&lh_sweep_counts[0], 1ull);
+                atomicAdd(&lh_sweep_counts[1], (unsigned long long)__popc(act));
+                atomicAdd(&lh_sweep_counts[2], (unsigned long long)cnt_cand);
+                atomicAdd(&lh_sweep_counts[3], (unsigned long long)cnt_form);
+                atomicAdd(&lh_sweep_counts[4], (unsigned long long)cnt_need);
+                atomicAdd(&lh_sweep_counts[5], (unsigned long long)cnt_below);
+                atomicAdd(&lh_sweep_counts[6], (unsigned long long)__popc(pending));
+                atomicAdd(&lh_sweep_counts[7], (unsigned long long)cnt_class);
+            }
+        }
+#endif
         while (pending) {
             const int src = __ffs(pending) - 1;
             pending &= pending - 1;
@@ -982,4 +1025,21 @@ extern "C" lh_status lh_search_amax(const void* W, lh_dtype w_dtype, int64_t n_m
     if (n_mult < 1 || n_mult > 4096) return fail(LH_ERR_INVALID_ARG, "n_mult must be in [1, 4096]");
     return launch_sweep(W, w_dtype, n_mats, c_out, c_in, ld_w, global_amax, H, best_amax, best_code, true, start, step,
                         (int)n_mult, nullptr, 0, stream);
+}
+
+extern "C" lh_status lh_debug_sweep_counts(uint64_t* out, int clear) {
+    using namespace lh;
+    clear_error();
+#if LH_SWEEP_COUNTERS
+    if (clear) {
+        const unsigned long long z[8] = {};
+        return cuda_status(cudaMemcpyToSymbol(lh_sweep_counts, z, sizeof(z)), "clear sweep counts");
+    }
+    if (!out) return fail(LH_ERR_INVALID_ARG, "null out");
+    return cuda_status(cudaMemcpyFromSymbol(out, lh_sweep_counts, sizeof(unsigned long long) * 8), "read sweep counts");
+#else
+    (void)out;
+    (void)clear;
+    return fail(LH_ERR_UNSUPPORTED, "this library is built without the sweep's work counters");
+#endif
 }

@@ -206,3 +206,8 @@ def test_fma_probe_rejects_bad_arguments():
     assert lh.lh_probe_fma_flop(0, 10) == 0
     for packed, blocks, iters, out in [(1, 0, 10, FAKE), (0, 10, 0, FAKE), (1, 10, 10, 0), (0, 1 << 21, 10, FAKE)]:
         assert lh.lh_probe_fma(packed, blocks, iters, out, stream=0, check=False) == 1
+
+
+def test_sweep_counts_only_in_the_measurement_build():
+    lh = _lh()
+    assert lh._binding.lib().lh_debug_sweep_counts(None, 1) == 2  # LH_ERR_UNSUPPORTED, no device call
