@@ -18,7 +18,9 @@ split over ranks is a MAX all-reduce. Total work is fixed (strong scaling).
 
 Prints one JSON line (rank 0). `value` is NVFP4 blocks calibrated per second of
 the whole step over all ranks. Timing: CUDA events on the launching stream, L2
-flushed (a 256 MB write) before every timed step, max over ranks.
+flushed before every timed step (a 256 MB write, then a 256 MB read of another
+buffer, so that the lines the flush wrote are written back before the step
+rather than during it), max over ranks.
 `--impl reference` times the FP64 CPU oracle on the host cores on bounded
 samples of the same layer, extrapolated to it (labelled so in the line).
 """
@@ -162,7 +164,8 @@ def parallelism_desc(ws: int) -> str:
 def bench_config(layer, ws: int) -> dict:
     """The `config` of the JSON line; the same dict on both arms."""
     return dict(workload=workload_desc(layer), blocks=int(layer.n_blocks), tokens=int(layer.n_tok),
-                l2="flushed (256 MB write before every timed step)", parallelism=parallelism_desc(ws))
+                l2="flushed before every timed step (256 MB write, then 256 MB read of another buffer)",
+                parallelism=parallelism_desc(ws))
 
 
 def spawn_ranks(args) -> int:
@@ -303,10 +306,10 @@ def sweep_work(lh, torch, dev, s, W, n_mats, c_out, c_in, ld, amax, H, codes, t_
     st = lib.lh_sweep_scales_ws(W.data_ptr(), dt, n_mats, c_out, c_in, ld, amax.data_ptr(), H.data_ptr(),
                                 a2.data_ptr(), c2.data_ptr(), wsp.data_ptr(), wsb, s)
     torch.cuda.synchronize(dev)
-    cnt = (ctypes.c_uint64 * 8)()
+    cnt = (ctypes.c_uint64 * 9)()
     if st != 0 or lib.lh_debug_sweep_counts(cnt, 0) != 0:
         return None
-    chunks, blocks, cand, forms, need, below, resweep, classes = (int(x) for x in cnt)
+    chunks, blocks, cand, forms, need, below, resweep, classes, pairs = (int(x) for x in cnt)
     if blocks == 0:
         return None
     fpb = 32.0 * forms / blocks
@@ -315,7 +318,8 @@ def sweep_work(lh, torch, dev, s, W, n_mats, c_out, c_in, ld, amax, H, codes, t_
     tf = flop * blocks / (t_sweep_ms / 1e3) / 1e12
     return dict(forms_per_block=fpb, lane_needed_forms_per_block=need / blocks,
                 candidates_quantised_per_block=qpb, class_bound_tests_per_block=32.0 * below / blocks,
-                fp64_resweeps_per_1000_blocks=1000.0 * resweep / blocks, flop_per_block=flop,
+                fp64_resweeps_per_1000_blocks=1000.0 * resweep / blocks,
+                fp64_pairs_per_1000_blocks=1000.0 * pairs / blocks, flop_per_block=flop,
                 achieved=tf, unit="TFLOP/s", frac=tf / fp32_peak, same_codes=bool(torch.equal(codes, c2)),
                 note="measurement build (liblh_counters.so): forms and candidates are counted per 32-lane warp, "
                      "so every lane pays for a form any lane needs; flop = 272 per form + 64 per quantised "
@@ -388,6 +392,13 @@ def run_ours(args):
     Wq = torch.empty(s_mats, s_out, s_cin, dtype=W.dtype, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 1 << 28) // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.zeros_like(flush)
+
+    def flush_l2():
+        """Cold L2: write a buffer twice its size, then read another one as large, so no
+        dirty line of the flush is left to be written back inside the timed region."""
+        flush.zero_()
+        flush_rd.amax()
     stream = torch.cuda.current_stream(dev)
     s = stream.cuda_stream
     ld = W.stride(1)
@@ -425,7 +436,7 @@ def run_ours(args):
 
     main = dict(W=W, X=X, off=off, amax=amax, H=H, ws=wsp, sws=swsp, codes=codes, bamax=bamax, Wq=Wq)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step_into(main, s)
     torch.cuda.synchronize(dev)
     assert n_loc == 0 or lh.lh_workspace_status(wsp, s) == 0
@@ -437,7 +448,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     sampler.start()
     for i in range(args.steps):
-        flush.zero_()  # cold L2 for every step
+        flush_l2()  # cold L2 for every step
         step_into(main, s, lambda k, e=evs[i]: e[k].record(stream))
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
@@ -484,7 +495,7 @@ def run_ours(args):
                 fn()
             ts = []
             for _ in range(reps):
-                flush.zero_()
+                flush_l2()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 fn()

@@ -142,10 +142,11 @@ LH_API int64_t lh_probe_fma_flop(int64_t blocks, int64_t iters);
 LH_API lh_status lh_probe_fma(int packed, int64_t blocks, int64_t iters, float* out, void* stream);
 
 /* Diagnostics; the pages have no counterpart. Work counters of the sweep,
- * summed over the launches since the last clear: out[8] = {warp chunks of 32
+ * summed over the launches since the last clear: out[9] = {warp chunks of 32
  * rows, blocks, candidates quantised per warp, full quadratic forms evaluated
  * per warp, forms some lane needed (lane count), class-wide bound tests, blocks
- * re-swept in FP64, mantissa classes walked per warp}. clear != 0 zeroes them
+ * re-swept in FP64 (all 126 codes), mantissa classes walked per warp, blocks
+ * whose best two candidates were compared in FP64}. clear != 0 zeroes them
  * (out unused). Only a library built with -DLH_SWEEP_COUNTERS=1 (the
  * measurement build, liblh_counters.so) counts; the library itself returns
  * LH_ERR_UNSUPPORTED. Synchronous. */

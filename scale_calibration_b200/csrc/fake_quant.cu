@@ -220,7 +220,7 @@ extern "C" lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, 
     const int sms = sm_count();
     if (sms <= 0) return fail(LH_ERR_CUDA, "no CUDA device");
     int64_t per = (rows + 7) / 8;  // 8 warps per CTA, one row per warp per pass
-    int64_t cap = ((int64_t)sms * 8 + n_mats - 1) / n_mats;
+    int64_t cap = ((int64_t)sms * 8) / n_mats;  // one wave of 8 CTAs per SM, none left over
     if (cap < 1) cap = 1;
     if (per > cap) per = cap;
     cudaLaunchConfig_t cfg = {};

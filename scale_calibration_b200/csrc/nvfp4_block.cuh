@@ -1,6 +1,6 @@
 // One NVFP4 block (16 weights) quantised with its chosen scale: the fake-quantised
 // values fp32(q * s), q = E2M1_RNE_sat(fp32(w / s)), and the packed 4-bit codes.
-// Shared by the fake-quant kernel and the sweep's fused epilogue (internal header).
+// Used by the fake-quant and packed-export kernel (internal header).
 //
 // "NVIDIA Model Optimizer Local-Hessian: 基于局部 Hessian 的 NVFP4 逐块权重缩放
 // 算法实战指南" (xxmr.cn/news/266017), section "算法原理": Q(W, s) = Cast(W/s) * s.
@@ -77,31 +77,50 @@ __device__ __forceinline__ float2 e2m1x2_values(uint32_t codes) {
 // fp32(w / s) for the 16 weights, then the E2M1 codes and values. The quotient is
 // formed from one correctly rounded reciprocal y = RN(1/s): q = RN(w y), r = w - s q
 // (exact, one FMA), RN(q + r y) is the correctly rounded quotient (P. Markstein,
-// IBM J. Res. Dev. 34(1), 1990) while s is normal and no non-zero |w| is below
-// 2^-100; other blocks divide. s == 0 gives q = +-0 with the sign of w.
+// IBM J. Res. Dev. 34(1), 1990) while s is normal and |w| >= 2^-100. With s in
+// [2^-95, FLT_MAX] a weight below 2^-100 has |w / s| < 2^-5: the approximate quotient
+// stays below 2^-4 as well, and both round to a zero of w's sign in E2M1, so one test
+// of s per block covers every weight. Other blocks divide; s == 0 gives q = +-0 with
+// the sign of w.
+//
+// The steps run on pairs (f32x2) with -y in place of y: a = RN(w (-y)) = -q,
+// r = RN(a s + w), v = RN(r (-y) + a) = -RN(q + r y), so v is the negated quotient
+// with the right sign even for w = +-0 (an FMA with a = -q keeps the zero's sign
+// that q + r y would lose). Its E2M1 codes get their sign bits flipped, and their
+// values are multiplied by -s.
 template <bool kOut, bool kPack>
 __device__ __forceinline__ void quantize_block(const float (&w)[16], float s, float (&o)[16], uint32_t (&word)[2]) {
-    float mn = __int_as_float(0x7F800000);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mn = (w[i] != 0.0f) ? fminf(mn, fabsf(w[i])) : mn;
-    const bool fast = s >= 1.17549435e-38f && mn >= 7.888609e-31f;
-    const float y = fast ? __frcp_rn(s) : 0.0f;
     word[0] = word[1] = 0u;
+    if (s >= 2.524355e-29f && s <= 3.4028235e38f) {  // 2^-95 <= s <= FLT_MAX
+        const float ny = -__frcp_rn(s);
+        const float2 ny2 = make_float2(ny, ny), s2 = make_float2(s, s), ns2 = make_float2(-s, -s);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const float2 w2 = make_float2(w[2 * p], w[2 * p + 1]);
+            const float2 a = __fmul2_rn(w2, ny2);
+            const float2 r = __ffma2_rn(a, s2, w2);
+            const float2 v = __ffma2_rn(r, ny2, a);
+            const uint32_t c2 = e2m1x2_codes(v.x, v.y);  // codes of -q, element 2p in the low nibble
+            if constexpr (kOut) {
+                const float2 q = __fmul2_rn(e2m1x2_values(c2), ns2);
+                o[2 * p] = q.x;
+                o[2 * p + 1] = q.y;
+            }
+            if constexpr (kPack) word[p >> 2] |= c2 << (8 * (p & 3));
+        }
+        word[0] ^= 0x88888888u;  // the sign bit of every nibble
+        word[1] ^= 0x88888888u;
+        return;
+    }
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
         float u[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const float wi = w[2 * p + h];
-            if (fast) {
-                const float q0 = __fmul_rn(wi, y);
-                // the last FMA turns -0 (w = -0) into +0; the quotient's sign is that of w
-                u[h] = copysignf(__fmaf_rn(__fmaf_rn(-q0, s, wi), y, q0), wi);
-            } else {
-                u[h] = (s != 0.0f) ? __fdiv_rn(wi, s) : copysignf(0.0f, wi);
-            }
+            u[h] = (s != 0.0f) ? __fdiv_rn(wi, s) : copysignf(0.0f, wi);
         }
-        const uint32_t c2 = e2m1x2_codes(u[0], u[1]);  // element 2p in the low nibble
+        const uint32_t c2 = e2m1x2_codes(u[0], u[1]);
         if constexpr (kOut) {
             const float2 q = e2m1x2_values(c2);
             o[2 * p] = __fmul_rn(q.x, s);

@@ -44,8 +44,9 @@
 #if LH_SWEEP_COUNTERS
 // [0] warp chunks, [1] blocks, [2] candidates quantised (per warp), [3] full forms (per
 // warp), [4] forms a lane needed (its bound did not exclude the candidate), [5] class-wide
-// bound tests, [6] blocks re-swept in FP64, [7] classes walked (per warp)
-__device__ unsigned long long lh_sweep_counts[8];
+// bound tests, [6] blocks re-swept in FP64, [7] classes walked (per warp), [8] blocks whose
+// best two were compared in FP64
+__device__ unsigned long long lh_sweep_counts[9];
 #endif
 
 #ifndef LH_SWEEP_UREGS
@@ -304,8 +305,10 @@ __device__ __forceinline__ float quad_form_smem(const float2 (&dw)[8], const Swe
 // subtracted to cover it. mu = 0 (no pruning) when H has a zero diagonal
 // entry with a non-zero off-diagonal entry in its row or a negative diagonal
 // entry, or when mu would fall below 2^-8.
-// Every thread of the CTA calls it (it holds __syncthreads); H is in sm.Hf.
-__device__ __forceinline__ void column_bounds(SweepShared& sm, int tid) {
+// Every thread of the CTA calls it (it holds __syncthreads); H is in sm.Hf. Sm is the
+// sweep's shared state or the bounds kernel's smaller one (Hf, pd, mu, nu).
+template <typename Sm>
+__device__ __forceinline__ void column_bounds(Sm& sm, int tid) {
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int hl = lane >> 4, i = lane & 15;
@@ -557,8 +560,11 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         unsigned cnt_cand = 0, cnt_form = 0, cnt_need = 0, cnt_below = 0, cnt_class = 0;
 #endif
         float best_e = __int_as_float(0x7F800000), second_e = __int_as_float(0x7F800000);
-        int best_fk = -1;  // 32 f + k of the best candidate (class f, step k); the code is formed at the end
-        bool flag = !fast;
+        float third_e = __int_as_float(0x7F800000);  // the smallest FP32 error after the best two
+        int best_fk = -1;    // 32 f + k of the best candidate (class f, step k); the code is formed at the end
+        int second_fk = -1;  // the same for the runner-up
+        bool flag = !fast;   // the whole block is re-swept in FP64
+        bool pair = false;   // only the best two are within the FP32 error bound: they are compared in FP64
         if (g == 0.0f) flag = false;  // every s_c is 0: q = 0, all errors equal, code 1
 
         if (fast) {
@@ -769,11 +775,17 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         if (!allowed(class_code(f, x0 + k), tid)) E = __int_as_float(0x7F800000);
                     }
                     if (E < best_e) {
+                        third_e = second_e;
                         second_e = best_e;
+                        second_fk = best_fk;
                         best_e = E;
                         best_fk = 32 * f + k;
+                    } else if (E < second_e) {
+                        third_e = second_e;
+                        second_e = E;
+                        second_fk = 32 * f + k;
                     } else {
-                        second_e = fminf(second_e, E);
+                        third_e = fminf(third_e, E);
                     }
                     return stop;
                 };
@@ -824,17 +836,36 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     k += up ? 1 : -1;
                 }
             }
-            // Exact FP32 ties (second == best) are flagged too, so the FP64 re-sweep applies
-            // the lowest-code rule.
-            const bool clear = rel ? (second_e * (1.0f - 4.0f * 5.9604645e-8f) > best_e * up_fac * (1.0f + rho))
-                                   : (second_e - best_e > margin);
-            if (!clear) flag = true;  // also catches NaN / inf
+            // A candidate whose FP32 error is clear of the best's by the error bound cannot be the
+            // argmin or tie it; every candidate the bounds excluded cannot either. So when the
+            // runner-up is not clear but all others are, the argmin is one of the best two, and
+            // FP64 errors of those two decide it (exact FP32 ties included: the lowest-code rule);
+            // when a third one is not clear either, the whole block is re-swept in FP64.
+            auto clear = [&](float e) {
+                return rel ? (e * (1.0f - 4.0f * 5.9604645e-8f) > best_e * up_fac * (1.0f + rho))
+                           : (e - best_e > margin);
+            };
+            if (!clear(second_e)) {                                      // also catches NaN / inf
+                if (clear(third_e) && best_fk >= 0 && second_fk >= 0) pair = true;
+                else flag = true;
+            }
         }
-        int best_c = 1;
-        if (best_fk >= 0) {
-            const int f = best_fk >> 5;
+        auto fk_code = [](int fk) {
+            const int f = fk >> 5;
             const int tz = (f == 0) ? 3 : (f == 4) ? 2 : (f == 2 || f == 6) ? 1 : 0;
-            best_c = class_code(f, -6 - tz + (best_fk & 31));
+            return class_code(f, -6 - tz + (fk & 31));
+        };
+        int best_c = best_fk >= 0 ? fk_code(best_fk) : 1;
+
+        // the best two of a block whose other candidates are clear, in FP64 by its own lane
+        if (__any_sync(0xFFFFFFFFu, pair && active)) {
+            if (pair && active) {
+                const int second_c = fk_code(second_fk);
+                const double e1 = candidate_error_f64(w, g, best_c, sm.Us);
+                const double e2 = candidate_error_f64(w, g, second_c, sm.Us);
+                // lexicographic (error, code) minimum; a NaN error never wins
+                if (e2 < e1 || (e2 == e1 && second_c < best_c) || (e1 != e1 && e2 == e2)) best_c = second_c;
+            }
         }
 
         // FP64 re-sweep of flagged blocks, one block at a time across the warp.
@@ -842,6 +873,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 #if LH_SWEEP_COUNTERS
         {
             const unsigned act = __ballot_sync(0xFFFFFFFFu, active);
+            const unsigned prs = __ballot_sync(0xFFFFFFFFu, pair && active);
             if (lane == 0) {
                 atomicAdd(&lh_sweep_counts[0], 1ull);
                 atomicAdd(&lh_sweep_counts[1], (unsigned long long)__popc(act));
@@ -851,6 +883,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 atomicAdd(&lh_sweep_counts[5], (unsigned long long)cnt_below);
                 atomicAdd(&lh_sweep_counts[6], (unsigned long long)__popc(pending));
                 atomicAdd(&lh_sweep_counts[7], (unsigned long long)cnt_class);
+                atomicAdd(&lh_sweep_counts[8], (unsigned long long)__popc(prs));
             }
         }
 #endif
@@ -889,10 +922,17 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 }
 
 // One CTA per block column (m, j): mu and nu of its H, the same computation the
-// sweep kernel does inline when it has no workspace.
+// sweep kernel does inline when it has no workspace. Its shared state is only what
+// the bounds need, so many CTAs fit an SM.
+struct BoundsShared {
+    float Hf[256];
+    int pd[16];
+    float mu, nu;
+};
+
 __global__ void __launch_bounds__(kThreads) sweep_bounds_kernel(const float* __restrict__ H,
                                                                 ColBounds* __restrict__ out) {
-    __shared__ __align__(16) SweepShared sm;
+    __shared__ __align__(16) BoundsShared sm;
     const int64_t col = blockIdx.x;
     const float* Hj = H ? H + col * 256 : nullptr;
     for (int i = threadIdx.x; i < 256; i += kThreads) sm.Hf[i] = Hj ? Hj[i] : ((i % 17 == 0) ? 1.0f : 0.0f);
@@ -1032,11 +1072,11 @@ extern "C" lh_status lh_debug_sweep_counts(uint64_t* out, int clear) {
     clear_error();
 #if LH_SWEEP_COUNTERS
     if (clear) {
-        const unsigned long long z[8] = {};
+        const unsigned long long z[9] = {};
         return cuda_status(cudaMemcpyToSymbol(lh_sweep_counts, z, sizeof(z)), "clear sweep counts");
     }
     if (!out) return fail(LH_ERR_INVALID_ARG, "null out");
-    return cuda_status(cudaMemcpyFromSymbol(out, lh_sweep_counts, sizeof(unsigned long long) * 8), "read sweep counts");
+    return cuda_status(cudaMemcpyFromSymbol(out, lh_sweep_counts, sizeof(unsigned long long) * 9), "read sweep counts");
 #else
     (void)out;
     (void)clear;

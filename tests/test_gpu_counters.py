@@ -37,9 +37,9 @@ def test_counting_build_matches_and_counts(cuda_ok):
     assert lib.lh_sweep_scales_ws(W.data_ptr(), lh.LH_BF16, 1, 700, 256, 256, amax.data_ptr(), H.data_ptr(),
                                   bam.data_ptr(), codes.data_ptr(), ws.data_ptr(), J * 16, s) == 0
     torch.cuda.synchronize()
-    cnt = (ctypes.c_uint64 * 8)()
+    cnt = (ctypes.c_uint64 * 9)()
     assert lib.lh_debug_sweep_counts(cnt, 0) == 0
-    chunks, blocks, cand, forms, need, below, resweep, classes = (int(x) for x in cnt)
+    chunks, blocks, cand, forms, need, below, resweep, classes, pairs = (int(x) for x in cnt)
     assert np.array_equal(codes.cpu().numpy(), res["codes"])
     assert blocks == 700 * J and classes == 8 * chunks
-    assert 0 < forms <= cand <= 126 * chunks and need <= 32 * forms and resweep <= blocks
+    assert 0 < forms <= cand <= 126 * chunks and need <= 32 * forms and resweep + pairs <= blocks

@@ -168,20 +168,24 @@ def test_signed_zero_weights_keep_their_sign(cuda_ok):
         assert np.array_equal(packed.cpu().numpy(), p_ref)
 
 
-def test_e2m1_ties_and_saturation_through_fake_quant_and_export(cuda_ok):
+@pytest.mark.parametrize("g", [1.0, 2.0 ** -95])
+def test_e2m1_ties_and_saturation_through_fake_quant_and_export(cuda_ok, g):
     # every E2M1 rounding tie, its FP32 neighbours, grid points, saturation, tiny values and
-    # signed zeros, at four block scales: W_q bits and packed bytes equal the oracle's
+    # signed zeros, at four block scales: W_q bits and packed bytes equal the oracle's.
+    # g = 2^-95 puts the block scales on both sides of 2^-95 (s = 2^-96 .. 2^-94), where
+    # the kernel switches between the reciprocal quotient and IEEE division.
     import scale_calibration_b200 as lh
-    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1, 1.5, 2, 3, 4, 6, 6.5, 7, 100, 1e-30, 0], np.float32)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1, 1.5, 2, 3, 4, 6, 6.5, 7, 100,
+                     1e-30, 2.0 ** -6, 0.02, 0], np.float32)
     vals = np.concatenate([ties, np.nextafter(ties, np.float32(0)), np.nextafter(ties, np.float32(1e9))])
     vals = np.concatenate([vals, -vals, [np.float32(-0.0)]]).astype(np.float32)
     n = ((len(vals) + 15) // 16) * 16
     Wn = np.zeros((1, 4, n), np.float32)
     Wn[0, :, :len(vals)] = vals
     for r, f in enumerate((1.0, 2.0, 0.5, 1.5)):
-        Wn[0, r] *= np.float32(f)
-    cd = np.repeat(np.array([0x38, 0x40, 0x30, 0x3C], np.uint8)[:, None], n // 16, axis=1)[None]  # s = f (g = 1)
-    amax = np.array([2688.0], np.float32)
+        Wn[0, r] *= np.float32(f * g)
+    cd = np.repeat(np.array([0x38, 0x40, 0x30, 0x3C], np.uint8)[:, None], n // 16, axis=1)[None]  # s = f g
+    amax = np.array([2688.0 * g], np.float32)
     W, A, C = (torch.from_numpy(a).cuda() for a in (Wn, amax, cd))
     out = torch.empty_like(W)
     pk = torch.zeros(1, 4, n // 2, dtype=torch.uint8, device="cuda")
