@@ -110,7 +110,7 @@ __device__ __forceinline__ float2 div_by_recip2(float2 a, float2 nb, float2 y) {
 
 // IEEE quotients w_i / s0 for blocks holding a tiny non-zero weight (rare;
 // kept out of line so the hot loop stays small).
-__device__ __noinline__ void quotients_ieee(const float (&w)[16], float s0, float2 (&u)[8]) {
+__device__ __forceinline__ void quotients_ieee(const float (&w)[16], float s0, float2 (&u)[8]) {
 #pragma unroll
     for (int p = 0; p < 8; ++p) u[p] = make_float2(__fdiv_rn(w[2 * p], s0), __fdiv_rn(w[2 * p + 1], s0));
 }
@@ -118,7 +118,8 @@ __device__ __noinline__ void quotients_ieee(const float (&w)[16], float s0, floa
 // FP64 error of candidate code c for block w (definition order of the method:
 // s = fp32(v(c) g), q = E2M1(fp32(w/s)), dw = q s - w exact, E = dw^T H dw),
 // the form taken over the packed upper triangle Us (H_aa, H_ab + H_ba in FP64).
-__device__ __noinline__ double candidate_error_f64(const float (&w)[16], float g, int c, const double* Us) {
+// w is read from shared memory, so no caller keeps its weights in local memory.
+__device__ __noinline__ double candidate_error_f64(const float* w, float g, int c, const double* Us) {
     const float s = __fmul_rn(e4m3_value(c), g);
     const double sd = (double)s;
     double dw[16];
@@ -206,7 +207,9 @@ struct ColBounds {
 static_assert(sizeof(ColBounds) == 16, "16-byte column records");
 
 struct SweepShared {
-    unsigned long long key[kTileRows];    // (bits of the heavy channels' max |w|) << 32 | local row
+    // (bits of the heavy channels' max |w|) << 32 | local row; after the sort, 16 weights per
+    // thread for the FP64 paths (kTileRows * 8 bytes = kThreads * 16 floats)
+    unsigned long long key[kTileRows];
     unsigned long long order[kTileRows];  // the same, grouped by sort bucket
     uint32_t hist[kSortBuckets];
     double Us[136];                     // H_aa, H_ab + H_ba (a < b) in FP64, packed upper triangle
@@ -672,15 +675,22 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                             // candidate has dw = 6 s_c sigma - w, so E = 36 s^2 sHs - 6 s (sHw + wHs) + wHw;
                             // an all-zero candidate has dw = -w, so E = wHw
                             double sHs = 0.0, sHw_wHs = 0.0, wHw = 0.0;
+                            // the weights go through this thread's slot in shared memory (the loops
+                            // index them at run time)
+                            float* const wt = reinterpret_cast<float*>(sm.key) + 16 * tid;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                *reinterpret_cast<float4*>(wt + 4 * i) =
+                                    make_float4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 #pragma unroll 1
                             for (int a = 0; a < 16; ++a) {
-                                const double wa = (double)w[a];
-                                const double sa = (w[a] > 0.0f) ? 1.0 : (w[a] < 0.0f ? -1.0 : 0.0);
+                                const double wa = (double)wt[a];
+                                const double sa = (wt[a] > 0.0f) ? 1.0 : (wt[a] < 0.0f ? -1.0 : 0.0);
                                 double tw = 0.0, ts = 0.0;  // sum_{b >= a} Us_ab w_b, Us_ab sigma_b
                                 for (int b = a; b < 16; ++b) {
                                     const double h = sm.Us[tri(a, b)];
-                                    tw = fma(h, (double)w[b], tw);
-                                    ts = fma(h, (w[b] > 0.0f) ? 1.0 : (w[b] < 0.0f ? -1.0 : 0.0), ts);
+                                    tw = fma(h, (double)wt[b], tw);
+                                    ts = fma(h, (wt[b] > 0.0f) ? 1.0 : (wt[b] < 0.0f ? -1.0 : 0.0), ts);
                                 }
                                 wHw = fma(wa, tw, wHw);
                                 sHs = fma(sa, ts, sHs);
@@ -857,12 +867,22 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         };
         int best_c = best_fk >= 0 ? fk_code(best_fk) : 1;
 
+        // the FP64 paths read the block's weights from this thread's slot in shared memory
+        float* const wst = reinterpret_cast<float*>(sm.key);
+        if ((pair || flag) && active) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float4*>(wst + 16 * tid + 4 * i) =
+                    make_float4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+        __syncwarp();
+
         // the best two of a block whose other candidates are clear, in FP64 by its own lane
         if (__any_sync(0xFFFFFFFFu, pair && active)) {
             if (pair && active) {
                 const int second_c = fk_code(second_fk);
-                const double e1 = candidate_error_f64(w, g, best_c, sm.Us);
-                const double e2 = candidate_error_f64(w, g, second_c, sm.Us);
+                const double e1 = candidate_error_f64(wst + 16 * tid, g, best_c, sm.Us);
+                const double e2 = candidate_error_f64(wst + 16 * tid, g, second_c, sm.Us);
                 // lexicographic (error, code) minimum; a NaN error never wins
                 if (e2 < e1 || (e2 == e1 && second_c < best_c) || (e1 != e1 && e2 == e2)) best_c = second_c;
             }
@@ -890,15 +910,12 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
         while (pending) {
             const int src = __ffs(pending) - 1;
             pending &= pending - 1;
-            float wv[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) wv[i] = __shfl_sync(0xFFFFFFFFu, w[i], src);
             double be = 0.0;
             int bc = 127;
             const int src_tid = (tid & ~31) + src;
             for (int c = lane + 1; c <= 126; c += 32) {
                 if (!allowed(c, src_tid)) continue;
-                const double e = candidate_error_f64(wv, g, c, sm.Us);
+                const double e = candidate_error_f64(wst + 16 * src_tid, g, c, sm.Us);
                 if (bc == 127 || e < be) { be = e; bc = c; }
             }
 #pragma unroll
