@@ -46,7 +46,7 @@ UNIT = "blocks/s"
 SWEEP_FLOP_PER_BLOCK = 126 * 152 * 2   # 16 dw FMA + 136 symmetric-form FMA per candidate
 FP32_LANES_PER_SM = 128
 # kernels of ours launched per call (counted in the timed region's gpu_launches)
-LAUNCHES = dict(absmax=2, hessian_plain=2, hessian_grouped=2, sweep_ws=2, fake_quant=1)  # Hessian: main + parts kernel
+LAUNCHES = dict(absmax=2, hessian_plain=1, hessian_grouped=1, sweep_ws=2, fake_quant=1)
 
 
 def profiled_traffic(kernel_src: str, summary: str):

@@ -91,13 +91,15 @@ LH_API lh_status lh_absmax(const void* W, lh_dtype w_dtype, int64_t n_mats, int6
  * H: device f32 [n_groups][c_in/16][16][16], read and written (H += ...):
  *   accumulation can be split over batches and resumed across calls.
  * workspace: device, at least lh_hessian_workspace_bytes(...) bytes, 256-byte
- *   aligned, owned by the caller; it holds a status word, per-CTA counters and
- *   the partial sums of the (slab, group) segments that several CTAs share.
+ *   aligned, owned by the caller; it holds a status word, and the partial sums
+ *   (with their ready flags) of the (slab, group) segments that several CTAs
+ *   share.
  *   Its size depends on n_tokens_total and c_in only, is at most about 5.3 MB,
  *   and its contents need no clearing between calls; it must not be shared by
  *   calls in flight at the same time.
  * Work split: one kernel launch; each CTA (two per SM) reads an equal share of
- *   X whatever the group sizes.
+ *   X whatever the group sizes. A CTA waits (bounded, 1 s) only for parts that
+ *   CTAs with lower block indices publish, which the GPU has started before it.
  * Numerics: bf16 products are exact in FP32; tensor-core FP32 accumulation
  *   over at most 128 tokens, then FP64 accumulation, FP32 partial sums where a
  *   segment spans several CTAs, summed in a fixed order (deterministic), and

@@ -32,17 +32,22 @@
 //    is the only one to add to those entries of H and adds its sum with
 //    vector reductions (red.global.add.v4.f32, no wait for H to load);
 //    otherwise it stores the sum as its part of the (slab, group) segment in
-//    the workspace. A second kernel, launched as a programmatic dependent,
-//    adds each split segment's parts in band order to H. The order of every
-//    sum is fixed, so H is deterministic; no CTA waits on another.
+//    the workspace. Each band but the segment's last publishes its part (per
+//    epilogue warp: a fence, then a flag set to the launch's generation); the
+//    last band, whose share of the segment is the first piece of its walk,
+//    adds the parts in band order after the rest of its work, when the
+//    earlier bands, which end with that segment, are done with it too, and
+//    adds the sum to H with one reduction. The order of every sum is fixed,
+//    so H is deterministic. A CTA waits only for CTAs of earlier bands (lower
+//    block indices, which the GPU starts first), each wait bounded.
 //  * Nothing in the workspace needs clearing between calls: the parts are
-//    written before they are read in every call, and the status word carries
-//    the call's 48-bit generation, so a stale value from an earlier call (or a
-//    fresh buffer) never matches it.
-//  * Every mbarrier wait is bounded (1 s of globaltimer); on expiry the kernel
-//    records LH_ERR_TIMEOUT in the workspace status word and the CTA winds
-//    down. Decreasing group offsets are recorded as LH_ERR_INVALID_ARG (the
-//    walk stays in bounds).
+//    written before their flags are set, and the flags and the status word
+//    carry the call's 48-bit generation, so a stale value from an earlier call
+//    (or a fresh buffer) never matches it.
+//  * Every wait is bounded (1 s of globaltimer); on expiry the kernel records
+//    LH_ERR_TIMEOUT in the workspace status word and the CTA winds down.
+//    Decreasing group offsets are recorded as LH_ERR_INVALID_ARG (the walk
+//    stays in bounds, and waits for parts stop once an error is recorded).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -98,17 +103,18 @@ constexpr Grid make_grid(int64_t n_tok, int64_t c_in, int64_t cap) {
     return gr;
 }
 
-// Workspace: [header: status word, generation of the last launch][parts:
-// [bands][slabs][2][8 blocks][16][16] FP32]. Parts exist only with several
-// bands (a layer no wider than the grid), so their count is bounded by twice
-// the grid size.
+// Workspace: [header: status word, generation of the last launch][flags:
+// [bands][slabs][2][4 epilogue warps] u64][parts: [bands][slabs][2][8 blocks]
+// [16][16] FP32]. Parts and flags exist only with several bands (a layer no
+// wider than the grid), so their count is bounded by twice the grid size.
 struct WsLayout {
-    size_t part_off, total;
+    size_t flag_off, part_off, total;
 };
 constexpr WsLayout ws_layout(const Grid& gr) {
     WsLayout w{};
     const size_t pairs = gr.bands > 1 ? (size_t)gr.bands * (size_t)gr.slabs : 0;
-    w.part_off = kHeaderBytes;
+    w.flag_off = kHeaderBytes;
+    w.part_off = w.flag_off + (sizeof(unsigned long long) * 2 * 4 * pairs + 255) / 256 * 256;
     w.total = w.part_off + sizeof(float) * kPartFloats * 2 * pairs;
     return w;
 }
@@ -153,6 +159,7 @@ struct KParams {
     float* H;            // [G][J][16][16], H +=
     unsigned long long* hdr;       // [0] status: gen << 16 | lh_status, written on error; [1] gen of the launch
     float* parts;                  // [bands][slabs][2][8][16][16]
+    unsigned long long* flags;     // [bands][slabs][2][4]: gen once an epilogue warp's rows of that part are written
     unsigned long long gen;        // this launch's generation, < 2^48
 };
 
@@ -170,6 +177,98 @@ __device__ __forceinline__ int64_t band_of(const KParams& p, int64_t t) {
 // else 1 (its last piece: only the segment's first band).
 __device__ __forceinline__ int64_t part_slot(const KParams& p, int64_t k, int64_t slab, int64_t seg_lo) {
     return (k * p.slabs + slab) * 2 + (seg_lo <= band_start(p, k) ? 0 : 1);
+}
+
+// The flag of epilogue warp q for a part slot (see part_slot).
+__device__ __forceinline__ unsigned long long* part_flag(const KParams& p, int64_t slot, int q) {
+    return p.flags + slot * 4 + q;
+}
+__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long* a) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned long long* a, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(v) : "memory");
+}
+// Records `code` for this launch unless an error of this launch is there already.
+__device__ void record_error(const KParams& p, int code) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(p.hdr);
+    const unsigned long long v = (p.gen << 16) | (unsigned long long)code;
+    while ((cur >> 16) != p.gen) {
+        const unsigned long long prev = atomicCAS(p.hdr, cur, v);
+        if (prev == cur) break;
+        cur = prev;
+    }
+}
+// The sum of a segment (group g, one slab) that bands b0..k share, formed by its
+// last band k at the end of its work: this warp's 32 rows of each earlier band's
+// part once that band has published them, then the parts added in band order in
+// FP64 (this band's own, in slot 0, last) and the sum added to H with one
+// reduction. Bands wait only for bands before them (lower block indices, running
+// or done). False when a wait gave up; `stopped` then says it was not a timeout.
+__device__ bool combine_parts(const KParams& p, int64_t g, int64_t slab, int64_t seg_lo, int64_t k, int q, int row,
+                              volatile int* abort_flag, bool& stopped) {
+    const int lane = threadIdx.x & 31;
+    const int64_t b0 = band_of(p, seg_lo);
+    // lane i waits for the part of band base + i, 32 bands per round
+    for (int64_t base = b0; base < k; base += 32) {
+        const int64_t kb = base + lane;
+        const unsigned long long* f = kb < k ? part_flag(p, part_slot(p, kb, slab, seg_lo), q) : p.hdr + 1;
+        const unsigned long long want = kb < k ? p.gen : ~0ull;  // lanes past the last band just read
+        const uint64_t t0 = global_ns();
+        for (uint32_t it = 0;; ++it) {
+            if (__all_sync(0xFFFFFFFFu, want == ~0ull || ld_acquire(f) == want)) break;
+            if ((it & 15) == 15) {
+                const bool stop =
+                    *abort_flag || (*reinterpret_cast<volatile unsigned long long*>(p.hdr) >> 16) == p.gen;
+                if (__any_sync(0xFFFFFFFFu, stop)) {
+                    stopped = true;
+                    return false;
+                }
+                if (__any_sync(0xFFFFFFFFu, global_ns() - t0 > kTimeoutNs)) {
+                    stopped = false;
+                    return false;
+                }
+            }
+        }
+    }
+    __syncwarp();  // the parts the other lanes acquired are visible to the whole warp from here
+    double t[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) t[c] = 0.0;
+    for (int64_t k0 = b0; k0 <= k; k0 += 4) {
+        float4 v[4][4];  // four parts' loads in flight, then added in band order
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (k0 + i <= k) {
+                const float4* src =
+                    reinterpret_cast<const float4*>(p.parts + part_slot(p, k0 + i, slab, seg_lo) * kPartFloats + row * 16);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) v[i][c] = __ldcg(src + c);
+            }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (k0 + i <= k) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    t[4 * c] += v[i][c].x;
+                    t[4 * c + 1] += v[i][c].y;
+                    t[4 * c + 2] += v[i][c].z;
+                    t[4 * c + 3] += v[i][c].w;
+                }
+            }
+    }
+    const int64_t jb = slab * 8 + (row >> 4);
+    if (jb < p.J) {
+        float* hrow = p.H + ((g * p.J + jb) * 16 + (row & 15)) * 16;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(hrow + 4 * c), "f"((float)t[4 * c]),
+                         "f"((float)t[4 * c + 1]), "f"((float)t[4 * c + 2]), "f"((float)t[4 * c + 3])
+                         : "memory");
+    }
+    return true;
 }
 
 // Token range of group g, clamped to [0, N]; an inverted range is empty.
@@ -253,9 +352,6 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
     // the set-up above overlaps the kernel before (programmatic launch); X, the
     // offsets, H and the workspace are touched only after it has finished
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    // the parts kernel may launch now: its CTAs wait on the device for this grid to finish
-    // (griddepcontrol.wait), so they start adding parts the moment the last CTA exits
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0 && b == 0) p.hdr[1] = p.gen;
 
     const int64_t band = b / p.sgroups, sg = b - band * p.sgroups;
@@ -399,6 +495,13 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
         double sum[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) sum[c] = 0.0;
+        // a segment whose last band this is: its part is in slot 0, the bands before add theirs;
+        // the sum is formed after this CTA's other work, when they are done with theirs. It is
+        // the group holding the band's first token, the same in every slab of the CTA.
+        bool pending = false;
+        int32_t pend_g = 0;
+        int64_t pend_lo = 0;
+        bool seen_err = false;  // a wait stopped because the CTA aborts or an error of this launch is recorded
         while (ok) {
             if (!warp_wait(smem_u32(&S.dfull[acc]), acc_phase, abort_flag)) { ok = false; break; }
             const StageDesc d = S.edesc[acc];
@@ -432,22 +535,39 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
                                      : "memory");
                 }
             } else {
-                // this band's part of a segment that several bands share; the parts kernel adds them
-                float4* part = reinterpret_cast<float4*>(p.parts + part_slot(p, band, d.slab, d.seg_lo) * kPartFloats +
-                                                         row * 16);
+                // this band's part of a segment that several bands share
+                const int64_t slot = part_slot(p, band, d.slab, d.seg_lo);
+                float4* part = reinterpret_cast<float4*>(p.parts + slot * kPartFloats + row * 16);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     __stcg(part + c, make_float4((float)sum[4 * c], (float)sum[4 * c + 1], (float)sum[4 * c + 2],
                                                  (float)sum[4 * c + 3]));
+                if (d.seg_hi > bt1) {
+                    // a later band adds it: publish this warp's rows of the part
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) st_release(part_flag(p, slot, q), p.gen);
+                } else {
+                    // the segment's last band: sum the parts at the end of this CTA's work
+                    pending = true;
+                    pend_g = d.g;
+                    pend_lo = d.seg_lo;
+                }
             }
 #pragma unroll
             for (int c = 0; c < 16; ++c) sum[c] = 0.0;
+        }
+        for (int64_t sl = sl0; ok && pending && sl < sl1; ++sl)
+            ok = combine_parts(p, pend_g, sl, pend_lo, band, q, row, abort_flag, seen_err);
+        if (!ok && seen_err) {
+            ok = true;  // stopped for an error that is recorded already: no timeout to report
+            *abort_flag = 1;
         }
     }
 
     if (!ok) {
         *abort_flag = 1;
-        atomicExch(p.hdr, (p.gen << 16) | (unsigned long long)LH_ERR_TIMEOUT);
+        record_error(p, LH_ERR_TIMEOUT);
     }
     __syncthreads();
     if (*abort_flag) {
@@ -458,62 +578,6 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
     }
     fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
-}
-
-// Adds the parts of every segment that several bands share to H. CTA (slab, k)
-// looks at band boundary k of one slab: the group holding tokens t_k - 1 and
-// t_k (t_k the first token of band k) crosses it; the CTA of the segment's
-// first crossing (the group starts in band k - 1) adds the parts of bands
-// k - 1 .. b1 in band order, four H entries per thread with up to eight parts'
-// loads in flight. Launched as a programmatic dependent of hessian_tc_kernel:
-// its CTAs wait for that grid to finish before reading.
-constexpr int kPartsThreads = 512;  // 128 rows x 4 column chunks of a slab
-__global__ void __launch_bounds__(kPartsThreads) hessian_parts_kernel(const KParams p) {
-    __shared__ int64_t s_lo, s_hi, s_g;
-    const int64_t slab = blockIdx.x;  // boundary 1 of every slab first: with one group, the only ones at work
-    const int64_t k = blockIdx.y + 1;
-    const int64_t tk = band_start(p, k);
-    const int lane = threadIdx.x & 31;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (threadIdx.x < 32) {
-        // the same walk as the producer's: the first group that holds token tk - 1
-        int64_t g = find_group(p, tk - 1, lane), lo = 0, hi = 0;
-        while (g < p.G) {
-            group_range(p, g, lo, hi);
-            if (hi > tk - 1) break;
-            ++g;
-        }
-        if (lane == 0) {
-            s_g = g;
-            s_lo = lo;
-            s_hi = hi;
-        }
-    }
-    __syncthreads();
-    const int64_t g = s_g, lo = s_lo, hi = s_hi;
-    // a segment that crosses boundary k and starts in band k - 1
-    if (g >= p.G || lo >= tk || hi <= tk || lo < band_start(p, k - 1)) return;
-    const int row = threadIdx.x >> 2, c4 = threadIdx.x & 3;
-    const int64_t jb = slab * 8 + (row >> 4);
-    if (jb >= p.J) return;
-    const int64_t b1 = band_of(p, hi - 1);
-    float4* h4 = reinterpret_cast<float4*>(p.H + ((g * p.J + jb) * 16 + (row & 15)) * 16) + c4;
-    const float4 h0 = *h4;
-    double t0 = h0.x, t1 = h0.y, t2 = h0.z, t3 = h0.w;
-    for (int64_t k0 = k - 1; k0 <= b1; k0 += 8) {
-        float4 v[8];  // eight parts' loads in flight, then added in band order
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (k0 + i <= b1)
-                v[i] = __ldcg(reinterpret_cast<const float4*>(p.parts + part_slot(p, k0 + i, slab, lo) * kPartFloats +
-                                                              row * 16) + c4);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (k0 + i <= b1) {
-                t0 += v[i].x; t1 += v[i].y; t2 += v[i].z; t3 += v[i].w;
-            }
-    }
-    *h4 = make_float4((float)t0, (float)t1, (float)t2, (float)t3);
 }
 
 // Diagnostics: the bounded wait of the kernel above, on an mbarrier that
@@ -671,6 +735,7 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     kp.H = H;
     kp.hdr = reinterpret_cast<unsigned long long*>(ws);
     kp.parts = reinterpret_cast<float*>(ws + wl.part_off);
+    kp.flags = reinterpret_cast<unsigned long long*>(ws + wl.flag_off);
     kp.gen = next_generation();
 
     static std::once_flag attr_once;
@@ -692,15 +757,7 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    s = cuda_status(cudaLaunchKernelEx(&cfg, hessian_tc_kernel, tmap, tmap16, kp), "hessian_tc_kernel launch");
-    if (s != LH_OK || gr.bands == 1) return s;
-    // the parts of segments that several bands share (a programmatic dependent as well)
-    cudaLaunchConfig_t cfg2 = cfg;
-    // one group (no offsets): only boundary 1 of each slab starts a segment, so one CTA per slab
-    cfg2.gridDim = dim3((unsigned)gr.slabs, offsets ? (unsigned)(gr.bands - 1) : 1u);
-    cfg2.blockDim = dim3(kPartsThreads);
-    cfg2.dynamicSmemBytes = 0;
-    return cuda_status(cudaLaunchKernelEx(&cfg2, hessian_parts_kernel, kp), "hessian_parts_kernel launch");
+    return cuda_status(cudaLaunchKernelEx(&cfg, hessian_tc_kernel, tmap, tmap16, kp), "hessian_tc_kernel launch");
 }
 
 // ---------------------------------------------------------------------------
