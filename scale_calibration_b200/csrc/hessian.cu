@@ -86,8 +86,12 @@ constexpr uint32_t kIdesc = (1u << 4)            // D format F32
 
 
 // The grid: `bands` teams of `sgroups` CTAs. With at most `cap` CTAs: one CTA
-// per slab and as many bands as fit (each at least one stage of tokens), or,
-// for layers with more slabs than CTAs, one band and runs of slabs.
+// per slab and as many bands as fit, or, for layers with more slabs than CTAs,
+// one band and runs of slabs. Bands start on whole 128-token tiles and hold at
+// least kMinBandTiles tiles each (fewer, longer bands when the layer is short):
+// a band of a few tiles pays the CTA's set-up and the sum of the parts for
+// little streaming, and a band edge inside a tile costs a short extra stage.
+constexpr int64_t kMinBandTiles = 4;
 struct Grid {
     int64_t slabs, sgroups, bands;
     int64_t ctas() const { return sgroups * bands; }
@@ -96,9 +100,13 @@ constexpr Grid make_grid(int64_t n_tok, int64_t c_in, int64_t cap) {
     Grid gr{};
     gr.slabs = (c_in + kSlab - 1) / kSlab;
     gr.sgroups = gr.slabs < cap ? gr.slabs : cap;
-    const int64_t by_cap = cap / gr.sgroups;
-    const int64_t by_tok = (n_tok + kStageTok - 1) / kStageTok;
-    gr.bands = by_cap < by_tok ? by_cap : by_tok;
+    const int64_t tiles = (n_tok + kStageTok - 1) / kStageTok;
+    int64_t bmax = cap / gr.sgroups;
+    if (bmax > tiles) bmax = tiles;
+    if (bmax < 1) bmax = 1;
+    int64_t per = (tiles + bmax - 1) / bmax;  // tiles of the longest band
+    if (per < kMinBandTiles) per = kMinBandTiles;
+    gr.bands = (tiles + per - 1) / per;
     if (gr.bands < 1) gr.bands = 1;
     return gr;
 }
@@ -163,8 +171,12 @@ struct KParams {
     unsigned long long gen;        // this launch's generation, < 2^48
 };
 
-// First token of band k (the bands split [0, N) as evenly as integers allow).
-__device__ __forceinline__ int64_t band_start(const KParams& p, int64_t k) { return p.N * k / p.bands; }
+// First token of band k: the bands split the 128-token tiles of [0, N) as evenly as
+// integers allow (band k starts at tile floor(tiles k / bands)).
+__device__ __forceinline__ int64_t band_start(const KParams& p, int64_t k) {
+    const int64_t tiles = (p.N + kStageTok - 1) / kStageTok;
+    return min(p.N, kStageTok * (tiles * k / p.bands));
+}
 // The band holding token t.
 __device__ __forceinline__ int64_t band_of(const KParams& p, int64_t t) {
     int64_t k = min(t * p.bands / p.N, p.bands - 1);

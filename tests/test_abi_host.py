@@ -121,7 +121,7 @@ def test_hessian_workspace_is_bounded_and_fits_the_noalloc_scratch():
     sizes = [lh.lh_hessian_workspace_bytes(n, c, g) for n in (1, 255, 4096, 1 << 20, (1 << 31) - 1)
              for c in (16, 2048, 4096, 17408, 40960, (1 << 31) - 16) for g in (1, 64, 65535)]
     assert 0 < max(sizes) <= (8 << 20)
-    assert lh.lh_hessian_workspace_bytes(1 << 20, 4096, 1) == lh.lh_hessian_workspace_bytes(4096, 4096, 64)
+    assert lh.lh_hessian_workspace_bytes(1 << 20, 4096, 1) == lh.lh_hessian_workspace_bytes(8192, 4096, 64)
     assert lh.lh_hessian_workspace_bytes(256, 128, 1) < lh.lh_hessian_workspace_bytes(2048, 128, 1)
     # a layer wider than the grid runs as one band: no parts at all
     assert lh.lh_hessian_workspace_bytes(4096, 128 * 400, 1) == 256
@@ -136,7 +136,7 @@ def test_workspace_size_grows_with_tokens_then_stays_bounded():
     lh = _lh()
     a = lh.lh_hessian_workspace_bytes(256, 128, 1)
     b = lh.lh_hessian_workspace_bytes(2048, 128, 1)
-    c = lh.lh_hessian_workspace_bytes(2048, 4096, 64)
+    c = lh.lh_hessian_workspace_bytes(8192, 4096, 64)
     d = lh.lh_hessian_workspace_bytes(16384, 4096, 1)
     assert 0 < a < b <= c == d
     assert lh.lh_hessian_workspace_bytes(100, 0, 1) == 0
