@@ -92,6 +92,9 @@ constexpr uint32_t kIdesc = (1u << 4)            // D format F32
 // a band of a few tiles pays the CTA's set-up and the sum of the parts for
 // little streaming, and a band edge inside a tile costs a short extra stage.
 constexpr int64_t kMinBandTiles = 4;
+// Grouped X: a group's run costs about half a stage beyond its tokens (its short last
+// stage and its flush), charged when the bands are cut.
+constexpr int64_t kGroupCost = 64;
 struct Grid {
     int64_t slabs, sgroups, bands;
     int64_t ctas() const { return sgroups * bands; }
@@ -167,28 +170,103 @@ struct KParams {
     float* H;            // [G][J][16][16], H +=
     unsigned long long* hdr;       // [0] status: gen << 16 | lh_status, written on error; [1] gen of the launch
     float* parts;                  // [bands][slabs][2][8][16][16]
-    unsigned long long* flags;     // [bands][slabs][2][4]: gen once an epilogue warp's rows of that part are written
+    unsigned long long* flags;     // [bands][slabs][2][4]: gen << 1 once an epilogue warp's rows of that part are
+                                   // written, gen << 1 | 1 when the band had no part to give (see combine_parts)
     unsigned long long gen;        // this launch's generation, < 2^48
+    int64_t gcost;                 // grouped X: tokens' worth of work charged per group when cutting bands
+    int64_t ctot;                  // N + gcost G: the total cost the bands share
 };
 
-// First token of band k: the bands split the 128-token tiles of [0, N) as evenly as
-// integers allow (band k starts at tile floor(tiles k / bands)).
-__device__ __forceinline__ int64_t band_start(const KParams& p, int64_t k) {
-    const int64_t tiles = (p.N + kStageTok - 1) / kStageTok;
-    return min(p.N, kStageTok * (tiles * k / p.bands));
+// For two costs T[0] <= T[1]: the first g in [0, G) whose group end, with gcost
+// charged for it and every group before it, reaches T[i]: hi_g + gcost (g + 1) >=
+// T[i] (hi_g = offsets[g + 1] clamped to [0, N]); G when none. Both searches by the
+// whole warp, step by step together (32 probes each per step, two steps for
+// G <= 1024). Exact for non-decreasing offsets; bounded answers in [0, G] for any
+// others.
+__device__ void find_band_groups(const KParams& p, const int64_t (&T)[2], int64_t (&out)[2], int lane) {
+    auto key = [&](int64_t g) { return min(max(__ldg(p.off + g + 1), (int64_t)0), p.N) + p.gcost * (g + 1); };
+    int64_t lo[2] = {0, 0}, n[2] = {p.G, p.G};
+    bool done[2] = {false, false};
+    while (!(done[0] && done[1])) {
+        int64_t ak[2];
+        bool hit[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int64_t step = n[i] > 32 ? (n[i] + 31) / 32 : 1;
+            ak[i] = min(lo[i] + (int64_t)(lane + 1) * step - 1, lo[i] + n[i] - 1);
+            hit[i] = !done[i] && (n[i] > 32 || lane < n[i]) && key(ak[i]) >= T[i];  // loads of both in flight
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const unsigned m = __ballot_sync(0xFFFFFFFFu, hit[i]);
+            if (done[i]) continue;
+            if (n[i] <= 32) {
+                out[i] = m ? lo[i] + __ffs(m) - 1 : lo[i] + n[i];
+                done[i] = true;
+            } else if (m == 0) {
+                out[i] = lo[i] + n[i];
+                done[i] = true;
+            } else {
+                const int64_t step = (n[i] + 31) / 32;
+                const int k = __ffs(m) - 1;
+                const int64_t nlo = lo[i] + (int64_t)k * step;
+                n[i] = min(lo[i] + (int64_t)(k + 1) * step - 1, lo[i] + n[i] - 1) - nlo + 1;
+                lo[i] = nlo;
+            }
+        }
+    }
 }
-// The band holding token t.
-__device__ __forceinline__ int64_t band_of(const KParams& p, int64_t t) {
-    int64_t k = min(t * p.bands / p.N, p.bands - 1);
-    while (k + 1 < p.bands && band_start(p, k + 1) <= t) ++k;
-    while (k > 0 && band_start(p, k) > t) --k;
-    return k;
+
+// Cost threshold of band k's first token: T_k = floor(ctot k / bands).
+__device__ __forceinline__ int64_t band_cost(const KParams& p, int64_t k) { return p.ctot * k / p.bands; }
+
+// First token of bands k and k + 1 (warp-wide: every lane calls it), and a group at
+// or before the one holding band k's first token. One group: the 128-token tiles of
+// [0, N) split as evenly as integers allow (band k starts at tile floor(tiles k /
+// bands)). Groups: each group's run ends in a short stage and a flush, so a group is
+// charged gcost tokens' worth of work, and band k starts at the first token t whose
+// cost, t + gcost (groups ending at or before t), reaches T_k; a band edge that falls
+// on a group's end starts the next group whole.
+__device__ void band_range(const KParams& p, int64_t k, int lane, int64_t& t0, int64_t& t1, int64_t& g0) {
+    g0 = 0;
+    if (!p.off) {
+        const int64_t tiles = (p.N + kStageTok - 1) / kStageTok;
+        t0 = k <= 0 ? 0 : min(p.N, kStageTok * (tiles * k / p.bands));
+        t1 = k + 1 >= p.bands ? p.N : min(p.N, kStageTok * (tiles * (k + 1) / p.bands));
+        return;
+    }
+    const int64_t T[2] = {band_cost(p, k), band_cost(p, k + 1)};
+    int64_t g[2];
+    find_band_groups(p, T, g, lane);
+    int64_t t[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        if (g[i] >= p.G) {
+            t[i] = T[i] - p.gcost * p.G;
+        } else {
+            // tokens of group g cost t + gcost g, and its end costs hi_g + gcost (g + 1) >= T
+            const int64_t hi = min(max(__ldg(p.off + g[i] + 1), (int64_t)0), p.N);
+            t[i] = min(T[i] - p.gcost * g[i], hi);
+        }
+        t[i] = min(max(t[i], (int64_t)0), p.N);
+    }
+    t0 = k <= 0 ? 0 : t[0];
+    t1 = k + 1 >= p.bands ? p.N : t[1];
+    g0 = k <= 0 ? 0 : min(g[0], p.G);
 }
-// Slot of band k's part of a segment that starts at token seg_lo: 0 when the
-// segment holds the band's first token (the band's first piece of the slab),
-// else 1 (its last piece: only the segment's first band).
-__device__ __forceinline__ int64_t part_slot(const KParams& p, int64_t k, int64_t slab, int64_t seg_lo) {
-    return (k * p.slabs + slab) * 2 + (seg_lo <= band_start(p, k) ? 0 : 1);
+// The first band of the segment of group g that starts at token seg_lo (its first
+// token, so the groups ending at or before it are g's predecessors): the last band
+// whose T_k is at most the cost seg_lo + gcost g. Exact for non-decreasing offsets.
+__device__ __forceinline__ int64_t first_band(const KParams& p, int64_t g, int64_t seg_lo) {
+    if (!p.off) return 0;
+    const int64_t c = seg_lo + p.gcost * g;
+    return max((int64_t)0, min(p.bands - 1, ((c + 1) * p.bands - 1) / p.ctot));
+}
+// Part slot of band k in one slab: s = 0 for a segment that began in an earlier band
+// (the band's first piece), s = 1 for one that begins in this band and goes on into
+// the next (its last piece).
+__device__ __forceinline__ int64_t part_slot(const KParams& p, int64_t k, int64_t slab, int s) {
+    return (k * p.slabs + slab) * 2 + s;
 }
 
 // The flag of epilogue warp q for a part slot (see part_slot).
@@ -215,22 +293,50 @@ __device__ void record_error(const KParams& p, int code) {
 }
 // The sum of a segment (group g, one slab) that bands b0..k share, formed by its
 // last band k at the end of its work: this warp's 32 rows of each earlier band's
-// part once that band has published them, then the parts added in band order in
-// FP64 (this band's own, in slot 0, last) and the sum added to H with one
-// reduction. Bands wait only for bands before them (lower block indices, running
+// part once that band has published them (band b0's in slot 1, the others' in slot
+// 0; a band that held no tokens publishes an empty flag), then the parts added in
+// band order in FP64 (this band's own, in slot 0, last) and the sum added to H with
+// one reduction. Bands wait only for bands before them (lower block indices, running
 // or done). False when a wait gave up; `stopped` then says it was not a timeout.
 __device__ bool combine_parts(const KParams& p, int64_t g, int64_t slab, int64_t seg_lo, int64_t k, int q, int row,
                               volatile int* abort_flag, bool& stopped) {
     const int lane = threadIdx.x & 31;
-    const int64_t b0 = band_of(p, seg_lo);
-    // lane i waits for the part of band base + i, 32 bands per round
+    const int64_t b0 = first_band(p, g, seg_lo);
+    double t[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) t[c] = 0.0;
+    auto add_parts = [&](const int64_t (&kb)[4], int n) {
+        float4 v[4][4];  // up to four parts' loads in flight, then added in band order
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (i < n) {
+                const float4* src = reinterpret_cast<const float4*>(
+                    p.parts + part_slot(p, kb[i], slab, kb[i] == b0 ? 1 : 0) * kPartFloats + row * 16);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) v[i][c] = __ldcg(src + c);
+            }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (i < n) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    t[4 * c] += v[i][c].x;
+                    t[4 * c + 1] += v[i][c].y;
+                    t[4 * c + 2] += v[i][c].z;
+                    t[4 * c + 3] += v[i][c].w;
+                }
+            }
+    };
+    // bands base .. base + 31 at a time: lane i waits for the flag of band base + i
     for (int64_t base = b0; base < k; base += 32) {
         const int64_t kb = base + lane;
-        const unsigned long long* f = kb < k ? part_flag(p, part_slot(p, kb, slab, seg_lo), q) : p.hdr + 1;
-        const unsigned long long want = kb < k ? p.gen : ~0ull;  // lanes past the last band just read
+        const unsigned long long* f =
+            kb < k ? part_flag(p, part_slot(p, kb, slab, kb == b0 ? 1 : 0), q) : p.hdr + 1;
         const uint64_t t0 = global_ns();
+        unsigned long long v = 0;
         for (uint32_t it = 0;; ++it) {
-            if (__all_sync(0xFFFFFFFFu, want == ~0ull || ld_acquire(f) == want)) break;
+            if (kb < k) v = ld_acquire(f);
+            if (__all_sync(0xFFFFFFFFu, kb >= k || (v >> 1) == p.gen)) break;
             if ((it & 15) == 15) {
                 const bool stop =
                     *abort_flag || (*reinterpret_cast<volatile unsigned long long*>(p.hdr) >> 16) == p.gen;
@@ -244,32 +350,21 @@ __device__ bool combine_parts(const KParams& p, int64_t g, int64_t slab, int64_t
                 }
             }
         }
+        __syncwarp();  // the parts the other lanes acquired are visible to the whole warp from here
+        unsigned have = __ballot_sync(0xFFFFFFFFu, kb < k && (v & 1ull) == 0);  // bands with a part
+        while (have) {
+            int64_t kbs[4];
+            int n = 0;
+            while (have && n < 4) {
+                kbs[n++] = base + __ffs(have) - 1;
+                have &= have - 1;
+            }
+            add_parts(kbs, n);
+        }
     }
-    __syncwarp();  // the parts the other lanes acquired are visible to the whole warp from here
-    double t[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) t[c] = 0.0;
-    for (int64_t k0 = b0; k0 <= k; k0 += 4) {
-        float4 v[4][4];  // four parts' loads in flight, then added in band order
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (k0 + i <= k) {
-                const float4* src =
-                    reinterpret_cast<const float4*>(p.parts + part_slot(p, k0 + i, slab, seg_lo) * kPartFloats + row * 16);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) v[i][c] = __ldcg(src + c);
-            }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (k0 + i <= k) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    t[4 * c] += v[i][c].x;
-                    t[4 * c + 1] += v[i][c].y;
-                    t[4 * c + 2] += v[i][c].z;
-                    t[4 * c + 3] += v[i][c].w;
-                }
-            }
+    {
+        const int64_t own[4] = {k, k, k, k};
+        add_parts(own, 1);
     }
     const int64_t jb = slab * 8 + (row >> 4);
     if (jb < p.J) {
@@ -290,36 +385,23 @@ __device__ __forceinline__ void group_range(const KParams& p, int64_t g, int64_t
     hi = min(max(__ldg(p.off + g + 1), lo), p.N);
 }
 
-// First group g whose offsets[g + 1] exceeds token t (G when none), by the whole
-// warp: each step probes 32 evenly spaced offsets at once (two steps for G <= 1024).
-// Exact for non-decreasing offsets; a bounded answer in [0, G] for any others.
-__device__ int64_t find_group(const KParams& p, int64_t t, int lane) {
-    if (!p.off) return 0;
-    int64_t lo = 0, n = p.G;
-    while (n > 32) {
-        const int64_t step = (n + 31) / 32;
-        const int64_t ak = min(lo + (int64_t)(lane + 1) * step - 1, lo + n - 1);
-        const unsigned m = __ballot_sync(0xFFFFFFFFu, __ldg(p.off + ak + 1) > t);
-        if (m == 0) return lo + n;
-        const int k = __ffs(m) - 1;
-        const int64_t nlo = lo + (int64_t)k * step;
-        n = min(lo + (int64_t)(k + 1) * step - 1, lo + n - 1) - nlo + 1;
-        lo = nlo;
-    }
-    const unsigned m = __ballot_sync(0xFFFFFFFFu, lane < n && __ldg(p.off + lo + lane + 1) > t);
-    return m ? lo + __ffs(m) - 1 : lo + n;
-}
-
 // One stage as the producer hands it to the MMA warp and, through it, to the
 // epilogue.
 struct StageDesc {
     int32_t ntok;     // tokens of the stage (1..128); 0 marks the end of the CTA's work
-    int32_t flags;    // bit 0: last stage of its piece (flush)
+    int32_t flags;    // bit 0: last stage of its piece (flush); bits 1-2: the piece's role (kOwned ..
+                      // kLastBand); on the end marker, bit 3: the band holds no token
     int32_t slab;
     int32_t g;
     int64_t seg_lo;   // the group's first token (clamped): its segment in this slab is
     int64_t seg_hi;   // [seg_lo, seg_hi)
 };
+
+// What the end of a piece does with its sum: the group's tokens of the slab lie in
+// this band alone (add to H); the segment began in an earlier band and goes on into a
+// later one (part in slot 0, published); it begins here and goes on (slot 1,
+// published); it began earlier and ends here (slot 0; this band sums the parts).
+enum PieceRole : int32_t { kOwned = 0, kMiddle = 1, kFirstBand = 2, kLastBand = 3 };
 
 struct Smem {
     uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], dfull[2];
@@ -367,8 +449,7 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
     if (threadIdx.x == 0 && b == 0) p.hdr[1] = p.gen;
 
     const int64_t band = b / p.sgroups, sg = b - band * p.sgroups;
-    const int64_t bt0 = band_start(p, band), bt1 = band_start(p, band + 1);  // this CTA's tokens
-    const int64_t sl0 = p.slabs * sg / p.sgroups, sl1 = p.slabs * (sg + 1) / p.sgroups;  // and slabs
+    const int64_t sl0 = p.slabs * sg / p.sgroups, sl1 = p.slabs * (sg + 1) / p.sgroups;  // this CTA's slabs
     bool ok = true;
 
     if (warp == 0) {
@@ -378,9 +459,11 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap16)) : "memory");
         int stage = 0;
         uint32_t phase = 0;
+        int64_t bt0, bt1, gb;  // this band's tokens, and a group at or before the one holding bt0
+        band_range(p, band, lane, bt0, bt1, gb);
         for (int64_t slab = sl0; ok && slab < sl1; ++slab) {
             int64_t t = bt0;
-            int64_t g = find_group(p, t, lane);
+            int64_t g = gb;
             while (ok && t < bt1) {
                 int64_t lo = 0, hi = 0;
                 while (g < p.G) {
@@ -391,13 +474,14 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
                 if (g >= p.G || lo >= bt1) break;  // no group holds the rest of the band
                 t = max(t, lo);
                 const int64_t t1 = min(hi, bt1);
+                const int32_t role = lo >= bt0 ? (hi <= bt1 ? kOwned : kFirstBand) : (hi <= bt1 ? kLastBand : kMiddle);
                 for (int64_t ts = t; ts < t1; ts += kStageTok) {
                     const int ntok = (int)min((int64_t)kStageTok, t1 - ts);
                     if (!warp_wait(smem_u32(&S.empty[stage]), phase ^ 1, abort_flag)) { ok = false; break; }
                     if (lane == 0) {
                         StageDesc& d = S.sdesc[stage];
                         d.ntok = ntok;
-                        d.flags = (ts + kStageTok >= t1) ? 1 : 0;
+                        d.flags = ((ts + kStageTok >= t1) ? 1 : 0) | (role << 1);
                         d.slab = (int32_t)slab;
                         d.g = (int32_t)g;
                         d.seg_lo = lo;
@@ -432,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
             if (warp_wait(smem_u32(&S.empty[stage]), phase ^ 1, abort_flag)) {
                 if (lane == 0) {
                     S.sdesc[stage].ntok = 0;
+                    S.sdesc[stage].flags = bt0 >= bt1 ? 8 : 0;
                     mbar_arrive(smem_u32(&S.full[stage]));
                 }
             } else {
@@ -514,10 +599,14 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
         int32_t pend_g = 0;
         int64_t pend_lo = 0;
         bool seen_err = false;  // a wait stopped because the CTA aborts or an error of this launch is recorded
+        bool empty_band = false;
         while (ok) {
             if (!warp_wait(smem_u32(&S.dfull[acc]), acc_phase, abort_flag)) { ok = false; break; }
             const StageDesc d = S.edesc[acc];
-            if (d.ntok == 0) break;
+            if (d.ntok == 0) {
+                empty_band = (d.flags & 8) != 0;
+                break;
+            }
             if (!warp_wait(smem_u32(&S.tfull[acc]), acc_phase, abort_flag)) { ok = false; break; }
             fence_after();
             uint32_t r[32];
@@ -535,7 +624,8 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
             const int64_t jb = (int64_t)d.slab * 8 + blk;
             const bool in_h = jb < p.J;
             float* hrow = p.H + (((int64_t)d.g * p.J + jb) * 16 + a) * 16;
-            if (d.seg_lo >= bt0 && d.seg_hi <= bt1) {
+            const int role = (d.flags >> 1) & 3;
+            if (role == kOwned) {
                 // the group's tokens of this slab are all in this band: no other CTA adds to
                 // these entries of H, so a reduction is one ordered addition, H = fp32(H + fp32(sum))
                 if (in_h) {
@@ -548,17 +638,17 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
                 }
             } else {
                 // this band's part of a segment that several bands share
-                const int64_t slot = part_slot(p, band, d.slab, d.seg_lo);
+                const int64_t slot = part_slot(p, band, d.slab, role == kFirstBand ? 1 : 0);
                 float4* part = reinterpret_cast<float4*>(p.parts + slot * kPartFloats + row * 16);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     __stcg(part + c, make_float4((float)sum[4 * c], (float)sum[4 * c + 1], (float)sum[4 * c + 2],
                                                  (float)sum[4 * c + 3]));
-                if (d.seg_hi > bt1) {
+                if (role != kLastBand) {
                     // a later band adds it: publish this warp's rows of the part
                     __threadfence();
                     __syncwarp();
-                    if (lane == 0) st_release(part_flag(p, slot, q), p.gen);
+                    if (lane == 0) st_release(part_flag(p, slot, q), p.gen << 1);
                 } else {
                     // the segment's last band: sum the parts at the end of this CTA's work
                     pending = true;
@@ -569,6 +659,9 @@ __global__ void __launch_bounds__(kThreads, 2) hessian_tc_kernel(const __grid_co
 #pragma unroll
             for (int c = 0; c < 16; ++c) sum[c] = 0.0;
         }
+        // a band without tokens tells the segment that spans it that it has no part
+        if (ok && empty_band && lane == 0)
+            for (int64_t sl = sl0; sl < sl1; ++sl) st_release(part_flag(p, part_slot(p, band, sl, 0), q), (p.gen << 1) | 1);
         for (int64_t sl = sl0; ok && pending && sl < sl1; ++sl)
             ok = combine_parts(p, pend_g, sl, pend_lo, band, q, row, abort_flag, seen_err);
         if (!ok && seen_err) {
@@ -749,6 +842,8 @@ extern "C" lh_status lh_accumulate_hessian(const void* X, lh_dtype x_dtype, int6
     kp.parts = reinterpret_cast<float*>(ws + wl.part_off);
     kp.flags = reinterpret_cast<unsigned long long*>(ws + wl.flag_off);
     kp.gen = next_generation();
+    kp.gcost = offsets ? kGroupCost : 0;
+    kp.ctot = n_tokens_total + kp.gcost * kp.G;
 
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;

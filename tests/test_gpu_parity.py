@@ -90,6 +90,26 @@ def test_hessian_many_ragged_groups(cuda_ok):
     assert np.all(Hg[[3, 10, 11]] == 0)
 
 
+def test_hessian_pile_of_empty_groups(cuda_ok):
+    # 48 empty groups at one offset: the bands charge every group a share of work, so
+    # several bands start at that token and hold none; the big group after it spans
+    # five bands whose parts its last band sums
+    import scale_calibration_b200 as lh
+    counts = [700, 40] + [0] * 48 + [3000, 5, 1200, 0, 0, 900]
+    G = len(counts)
+    layer = synth.make_layer(8, 256, int(sum(counts)), seed=33, n_mats=G, counts=counts)
+    _, X, off = gu.to_device(layer)
+    H = torch.zeros(G, 16, 16, 16, device="cuda")
+    wsb = lh.lh_hessian_workspace_bytes(layer.n_tok, 256, G)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    lh.lh_accumulate_hessian(X, lh.LH_BF16, layer.n_tok, 256, X.stride(0), off, G, H, ws, wsb)
+    assert lh.lh_workspace_status(ws) == 0
+    Hg = H.cpu().numpy()
+    per, whole, bad = gu.hessian_rel_errors(Hg, oracle.hessian(layer.X, c_in=256, offsets=layer.offsets))
+    assert per <= gu.HESSIAN_RTOL and whole <= gu.HESSIAN_RTOL and bad == 0, (per, whole, bad)
+    assert np.all(Hg[[c == 0 for c in counts]] == 0)
+
+
 def test_hessian_overlapping_offsets_are_reported(cuda_ok):
     # two groups over the same 1000 tokens hold more tiles than the workspace bound: the call
     # stays in bounds and the workspace status says the offsets are invalid
