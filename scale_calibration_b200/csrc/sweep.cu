@@ -217,6 +217,7 @@ struct SweepShared {
     float Ud[8];            // diagonals of the odd rows
     float Ua[136];          // |U| packed upper triangle, for the error bound
     float Hf[256];          // H as given, for the FP64 re-sweep
+    __align__(16) float chol[8][32];  // the Cholesky tests' columns, per half-warp (column bounds)
     float2 dg[8];           // diagonal of H, pairs (for the lower bound)
     int pd[16];             // results of the shifted positive-definiteness tests
     uint32_t allow[4][kThreads];  // amax search: the codes each thread's current block may take
@@ -231,9 +232,12 @@ struct SweepShared {
 };
 
 // Is C - mu I positive definite? FP32 Cholesky by one half-warp, in registers:
-// lane i (of 16) owns row i of C, and the multipliers of column k reach the
-// other rows by shuffles; true when every pivot is positive.
-__device__ __forceinline__ bool shifted_pd(const float (&crow)[16], float mu, int i) {
+// lane i (of 16) owns row i of C; the pivot of column k comes by a shuffle, and
+// the multipliers L_bk through `col`, this half-warp's 2 x 16 floats of shared
+// memory (one column per step, alternating, so one warp barrier a step suffices),
+// read back as 128-bit broadcasts; true when every pivot is positive. Every lane
+// of the warp calls it (the warp barriers).
+__device__ __forceinline__ bool shifted_pd(const float (&crow)[16], float mu, int i, float* col) {
     float c[16];
 #pragma unroll
     for (int b = 0; b < 16; ++b) c[b] = crow[b] - ((b == i) ? mu : 0.0f);
@@ -243,8 +247,17 @@ __device__ __forceinline__ bool shifted_pd(const float (&crow)[16], float mu, in
         const float d = __shfl_sync(0xFFFFFFFFu, c[k], k, 16);  // pivot, from lane k of this half
         ok = ok && (d > 0.0f);
         const float l = (i > k) ? c[k] * (d > 0.0f ? rsqrtf(d) : 1.0f) : 0.0f;  // L_ik
+        float* lk = col + 16 * (k & 1);
+        lk[i] = l;
+        __syncwarp();
 #pragma unroll
-        for (int b = k + 1; b < 16; ++b) c[b] = __fmaf_rn(-l, __shfl_sync(0xFFFFFFFFu, l, b, 16), c[b]);
+        for (int b4 = (k + 1) / 4 * 4; b4 < 16; b4 += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(lk + b4);
+            const float lb[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (b4 + u > k) c[b4 + u] = __fmaf_rn(-l, lb[u], c[b4 + u]);
+        }
     }
     return ok;
 }
@@ -342,7 +355,8 @@ __device__ __forceinline__ void column_bounds(Sm& sm, int tid) {
         if (tid == 0) sm.nu = rs * (1.0f + 1.5258789e-5f);
     }
     const float mu1 = 0.04f + 0.12f * (float)slot;
-    const bool ok1 = psd_rows && shifted_pd(crow, mu1, i);
+    float* const col = &sm.chol[slot][0];
+    const bool ok1 = psd_rows && shifted_pd(crow, mu1, i, col);
     if (i == 0) sm.pd[slot] = ok1;
     __syncthreads();
     float lo = 0.0f;
@@ -350,7 +364,8 @@ __device__ __forceinline__ void column_bounds(Sm& sm, int tid) {
         if (sm.pd[q]) lo = fmaxf(lo, 0.04f + 0.12f * (float)q);
     const float step = (lo > 0.0f ? 0.12f : 0.04f) * (1.0f / 9.0f);
     const float mu2 = lo + step * (float)(slot + 1);
-    const bool ok2 = psd_rows && shifted_pd(crow, mu2, i);
+    __syncwarp();  // the last step's reads of col are done
+    const bool ok2 = psd_rows && shifted_pd(crow, mu2, i, col);
     if (i == 0) sm.pd[8 + slot] = ok2;
     __syncthreads();
     float best = lo;
@@ -943,6 +958,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
 // the bounds need, so many CTAs fit an SM.
 struct BoundsShared {
     float Hf[256];
+    __align__(16) float chol[8][32];  // the Cholesky tests' columns, per half-warp
     int pd[16];
     float mu, nu;
 };
