@@ -19,7 +19,8 @@
 //    class consecutive codes double the scale exactly, so fp32(w / s_c) is
 //    fp32(w / s_c0) scaled by a power of two: 16 correctly rounded quotients
 //    per class replace 16 per candidate, and each candidate rounds them onto
-//    the E2M1 grid scaled by 2^k (exact).
+//    the E2M1 grid scaled by 2^k (exact: the quotients times 2^-k through the
+//    hardware E2M1 conversions, round to nearest even with saturation).
 //  * Per class a warp walks up and down from its max-scaling step. A lower
 //    bound mu * sum_a H_aa dw_a^2 <= E skips the form for candidates that
 //    cannot win, and class-wide bounds end each direction early; mu comes from
@@ -27,14 +28,16 @@
 //    a first kernel when the caller gives a workspace).
 //  * The survivors' E(c) is evaluated in FP32 with the symmetric form (136
 //    FMA). Its error is at most rho * E with rho = 48 u nu / mu (nu bounds the
-//    largest eigenvalue of |normalised H|), or an absolute bound when mu = 0;
-//    blocks whose runner-up is within that bound of the best are re-swept in
-//    FP64 by the whole warp. The result is the exact argmin (up to FP64
+//    largest eigenvalue of |normalised H|), or an absolute bound when mu = 0.
+//    When only the runner-up is within that bound of the best, the lane
+//    compares the two in FP64; when a third candidate is too, the whole warp
+//    re-sweeps the block in FP64. The result is the exact argmin (up to FP64
 //    rounding), lowest code on ties.
 #include <cmath>
 
 #include "common.cuh"
 #include "quant.cuh"
+#include <cuda_fp16.h>
 
 // Measurement build only (-DLH_SWEEP_COUNTERS=1): the work the walk does, summed
 // over a launch; lh_debug_sweep_counts reads and clears it. Off in the library.
@@ -102,6 +105,15 @@ __device__ __forceinline__ int class_code(int f, int x) {
 // while the remainder a - b q cannot underflow, i.e. for a >= 2^-100 (or a = 0)
 // and a normal b; blocks with a smaller non-zero |w| use IEEE division. The
 // packed FP32 operations round each lane exactly as the scalar ones; nb = -b.
+// Both values rounded to the nearest E2M1 value (ties to even, saturating at +-6),
+// by the hardware conversions: to two E2M1 codes, and back through f16x2 (exact).
+__device__ __forceinline__ float2 e2m1x2_round(float2 v) {
+    uint32_t h2;
+    asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}"
+        : "=r"(h2) : "f"(v.y), "f"(v.x));
+    const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+    return __half22float2(h);
+}
 __device__ __forceinline__ float2 div_by_recip2(float2 a, float2 nb, float2 y) {
     const float2 q = __fmul2_rn(a, y);
     const float2 r = __ffma2_rn(q, nb, a);
@@ -645,7 +657,6 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                 const float s0 = __fmul_rn(v0, g);
                 // signed quotients u = w / s0; candidate k of the class has the scale 2^k s0
                 float2 u[8];
-                unsigned ep[16];
                 float umax = 0.0f;  // max |u|
                 if (tiny_w) {
                     quotients_ieee(w, s0, u);
@@ -656,11 +667,7 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                     for (int p = 0; p < 8; ++p) u[p] = div_by_recip2(w2[p], ns02, rs02);
                 }
 #pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    ep[2 * p] = (__float_as_uint(u[p].x) & 0x7F800000u) + 0x0B400000u;
-                    ep[2 * p + 1] = (__float_as_uint(u[p].y) & 0x7F800000u) + 0x0B400000u;
-                    umax = fmaxf(umax, fmaxf(fabsf(u[p].x), fabsf(u[p].y)));
-                }
+                for (int p = 0; p < 8; ++p) umax = fmaxf(umax, fmaxf(fabsf(u[p].x), fabsf(u[p].y)));
                 const float2 ns0 = make_float2(-s0, -s0);
                 // One candidate; returns true (upward walk only) when every lane proves that no
                 // later candidate of the upward walk can beat the incumbent.
@@ -717,29 +724,20 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                         }
                     }
                     if (!done) {
-                        // q = RNE of u on the grid 2^k {0,.5,1,1.5,2,3,4,6,8,12,...}: the magic
-                        // constant M = 1.5 * 2^23 * spacing comes from the binade of |u|, raised to
-                        // that of 2^k; (u + M) - M rounds u to the spacing with ties to even (the
-                        // grid is symmetric, so the sign rides along). Values past 6 * 2^k land at
-                        // or beyond it and are clamped, in warps that hold any.
-                        float2 q[8];
-#pragma unroll
-                        for (int p = 0; p < 8; ++p) {
-                            const float2 M = make_float2(__uint_as_float(max(ep[2 * p], mlo)),
-                                                         __uint_as_float(max(ep[2 * p + 1], mlo)));
-                            q[p] = __ffma2_rn(M, make_float2(-1.0f, -1.0f), __fadd2_rn(u[p], M));  // exact
-                        }
+                        // q = 2^k E2M1_RNE_sat(u 2^-k): u 2^-k is exact (a power of two), and the
+                        // sm_100a conversions round it to nearest even on the E2M1 grid with
+                        // saturation at +-6 (two values per conversion) and give the values back
+                        // exactly through f16x2; dw takes the factor 2^k with -s0 2^k (exact).
                         const bool sat_any = __any_sync(0xFFFFFFFFu, umax > lim);
-                        if (sat_any) {
-#pragma unroll
-                            for (int p = 0; p < 8; ++p) {
-                                q[p].x = fminf(fmaxf(q[p].x, -lim), lim);
-                                q[p].y = fminf(fmaxf(q[p].y, -lim), lim);
-                            }
-                        }
+                        const float2 sck = make_float2(__int_as_float((127 - k) << 23), __int_as_float((127 - k) << 23));
+                        const float nsk = -s0 * __int_as_float((127 + k) << 23);  // -s0 2^k, exact
+                        const float2 nsk2 = make_float2(nsk, nsk);
                         float2 dw[8];
 #pragma unroll
-                        for (int p = 0; p < 8; ++p) dw[p] = __ffma2_rn(q[p], ns0, w2[p]);  // w - q_c s_c = -dw, one rounding
+                        for (int p = 0; p < 8; ++p) {
+                            const float2 uk = __fmul2_rn(u[p], sck);  // u 2^-k, exact
+                            dw[p] = __ffma2_rn(e2m1x2_round(uk), nsk2, w2[p]);  // w - q_c s_c = -dw, one rounding
+                        }
                         // E >= mu sum_a H_aa dw_a^2: skip the form when, for every lane, that bound
                         // (rounded down) exceeds the best so far by more than the FP32 error margin,
                         // so the candidate can neither be the argmin nor tie it
@@ -764,9 +762,12 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                                 // points in U = {0, .5, 1, 1.5, 2, 3, 4, 6, 8, 12, 16, ...} 2^k, so each
                                 // weight stays at least its distance to U away from it at every later
                                 // step. Below 6 * 2^k the nearest point of U is q here; above 4 * 2^k U is
-                                // the grid {1, 1.5} 2^m, to which the unclamped magic-constant rounding
-                                // goes, so |w - q s0| before the saturation clamp is that distance for
-                                // every weight (less 2^-23 |w| for the rounding of u).
+                                // the grid {1, 1.5} 2^m. When any weight saturates, the distances come
+                                // from an unclamped rounding onto U: the magic constant
+                                // M = 1.5 * 2^23 * spacing (spacing from the binade of |u|, at least that
+                                // of 2^k) makes (u + M) - M the round-to-nearest-even onto U (the grid
+                                // is symmetric, so the sign rides along), less 2^-23 |w| for the rounding
+                                // of u.
                                 float tail = lbraw;
                                 if (sat_any) {
                                     float2 tl2 = make_float2(0.0f, 0.0f);
@@ -776,8 +777,9 @@ sweep_kernel(const T* __restrict__ W, int64_t c_out, int64_t J, int64_t ld, int6
                                         float2 du[2];
 #pragma unroll
                                         for (int h = 0; h < 2; ++h) {
-                                            const float2 M = make_float2(__uint_as_float(max(ep[2 * (p + h)], mlo)),
-                                                                         __uint_as_float(max(ep[2 * (p + h) + 1], mlo)));
+                                            const unsigned ex = (__float_as_uint(u[p + h].x) & 0x7F800000u) + 0x0B400000u;
+                                            const unsigned ey = (__float_as_uint(u[p + h].y) & 0x7F800000u) + 0x0B400000u;
+                                            const float2 M = make_float2(__uint_as_float(max(ex, mlo)), __uint_as_float(max(ey, mlo)));
                                             const float2 qu = __ffma2_rn(M, make_float2(-1.0f, -1.0f), __fadd2_rn(u[p + h], M));
                                             du[h] = __ffma2_rn(qu, ns0, w2[p + h]);
                                         }
