@@ -203,9 +203,10 @@ LH_API lh_status lh_noalloc_status(void* stream);
  *   best_code[m][r][j] = argmin_c E(c)  (lowest code on ties)
  *   best_amax[m][r][j] = fp32(6 * s_best)
  *
- * E is evaluated in FP32; blocks whose two best candidates are closer than a
- * proven bound on the FP32 rounding error are re-evaluated in FP64, so the
- * chosen code is the exact argmin up to FP64 rounding.
+ * E is evaluated in FP32. When only the runner-up is within a proven bound on
+ * the FP32 rounding error of the best, the two are compared in FP64; when a
+ * third candidate is within it too, all 126 codes are re-evaluated in FP64. So
+ * the chosen code is the exact argmin up to FP64 rounding.
  * W: device bf16 or f32 [n_mats][c_out][ld_w]. global_amax: device f32 [n_mats], finite
  *   and >= 0 (as lh_absmax writes it); 0 is defined (every block gets code 1 and amax 0);
  *   a NaN, infinite or negative value is not detected and gives unspecified codes.
