@@ -339,6 +339,32 @@ def test_fake_quant_matches_independent_q_times_s():
             assert np.array_equal(out_bf[r, 16 * j:16 * j + 16], refb)
 
 
+@pytest.mark.parametrize("g", [1.0, 2.0 ** -95])
+def test_fake_quant_ties_at_tiny_and_unit_scales(g):
+    # every E2M1 tie and its FP32 neighbours, saturation, quotients below 2^-5 and signed
+    # zeros, at block scales f g for f in {1, 2, 0.5, 1.5}: the oracle equals the
+    # independent fp32(w / s) -> nearest E2M1 (ties to even) -> fp32(q s)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1, 1.5, 2, 3, 4, 6, 6.5, 7, 100,
+                     1e-30, 2.0 ** -6, 0.02, 0], np.float32)
+    vals = np.concatenate([ties, np.nextafter(ties, np.float32(0)), np.nextafter(ties, np.float32(1e9))])
+    vals = np.concatenate([vals, -vals, [np.float32(-0.0)]]).astype(np.float32)
+    n = ((len(vals) + 15) // 16) * 16
+    W = np.zeros((4, n), np.float32)
+    W[:, :len(vals)] = vals
+    for r, f in enumerate((1.0, 2.0, 0.5, 1.5)):
+        W[r] *= np.float32(f * g)
+    codes = np.repeat(np.array([0x38, 0x40, 0x30, 0x3C], np.uint8)[:, None], n // 16, axis=1)
+    A = np.float32(2688.0 * g)
+    out = oracle.fake_quant(W, [A], codes)
+    gs = oracle.global_scale(A)
+    ev = indep.e4m3_values_torch()
+    for r in range(4):
+        s = np.float32(np.float32(ev[codes[r, 0]]) * gs)
+        u = (W[r] / s).astype(np.float32)
+        ref = (indep.e2m1_nearest(u).astype(np.float32) * s).astype(np.float32)
+        assert np.array_equal(out[r].view(np.uint32), ref.view(np.uint32)), r
+
+
 def test_fake_quant_error_is_the_swept_dw():
     L = synth.make_layer(3, 32, 64, seed=17, w_dtype="f32")
     W = L.W_f32()[0]
